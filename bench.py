@@ -1,0 +1,422 @@
+"""Benchmark: semi-CRF forward+backward throughput on B200.
+
+One step = the whole hot path on one batch of synthetic input: centring and
+prefix scan, streaming forward (log Z + checkpoints), backward (checkpoint
+recompute, backward messages and marginals, gradient finalisation).  The
+metric is B*T*K*C segment-label updates per second (whole job over all ranks).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config ner]
+    python bench.py --impl reference ...   # the CPU oracle, same metric
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch (weak
+scaling) and the parameter gradients dA, dD are summed across ranks with an
+NCCL all-reduce inside the step.  Timing is CUDA events on the launching stream,
+max over ranks; L2 is flushed (256 MiB write) between timed steps.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import semicrf_workloads as wl  # noqa: E402
+
+METRIC = "semi-CRF fwd+bwd segment-label updates/sec (B·T·K·C/s), 1×B200, % roofline"
+UNIT = "updates/s"
+# B200: 148 SMs, 64 FP64 FMA lanes per SM per clock, 16 MUFU (SFU) lanes per SM per clock
+N_SM = 148
+FP64_FMA_PER_SM_CLK = 64
+MUFU_PER_SM_CLK = 16
+HBM_FALLBACK_GBS = 6650.0
+SM_MAX_MHZ_FALLBACK = 1965.0
+KERNEL_NAMES = ["scan_partials", "scan_offsets", "scan_apply", "fwd_kernel", "fwd_recompute",
+                "bwd_kernel", "finalise_params", "finalise_dx"]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return json.load(f)
+    except Exception:
+        return None
+
+
+def algorithmic(w):
+    """Terms and bytes the method must do (not the recompute it chooses to do)."""
+    sumL = int(w.lengths.astype(np.int64).sum())
+    terms_pass = sumL * (w.K * w.C + w.C * w.C)          # one (lse,+) term = one FMA in exp space
+    bytes_path = 4 * w.B * w.T * w.C * 2 + 8 * (w.C * w.C + w.K * w.C)
+    return sumL, terms_pass, bytes_path
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        q = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        mhz, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9 or (self.uuid and f[0] != self.uuid):
+                continue
+            try:
+                mhz.append(float(f[1]))
+                maxes.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def oracle_sample(w, budget_s=10.0, nthreads=0):
+    """Time the CPU oracle (forward + backward + gradients) on a bounded sample of
+    the workload: whole sequences, or a prefix of them when one is too slow."""
+    import oracle
+    nth = nthreads or os.cpu_count() or 1
+    # estimate: ~4 log-space exponentials per term, ~1.5e7 per second per thread
+    sumL, terms, _ = algorithmic(w)
+    est = 4 * terms / (1.5e7 * nth)
+    B, T = w.B, w.T
+    x, lengths = w.x, w.lengths
+    if est > budget_s:
+        # shrink: fewer sequences, then a shorter prefix of each
+        frac = budget_s / est
+        Bs = max(1, min(B, int(math.ceil(B * frac))))
+        Ts = T
+        if Bs == 1 and frac * B < 1:
+            Ts = max(w.K + 1, int(T * frac * B))
+        x = np.ascontiguousarray(w.x[:Bs, :Ts])
+        lengths = np.minimum(w.lengths[:Bs], Ts).astype(np.int32)
+        B, T = Bs, Ts
+    sample = f"B={B} of {w.B}, T={T} of {w.T}, K={w.K}, C={w.C}"
+    oracle.build()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.factorised(x, w.A, w.D, lengths, nthreads=nth)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 1000:
+            break
+    units = reps * B * T * w.K * w.C
+    return {"value": units / el, "unit": UNIT, "cores": nth, "kind": "oracle",
+            "sample": f"{sample}; {reps} repetition(s) in {el:.1f} s, float64 log-space, OpenMP"}
+
+
+# --------------------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import semi_markov_crf_prefix_b200 as sc
+    from semi_markov_crf_prefix_b200 import _lib
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    sc.load_library()
+
+    w = wl.make_workload(args.config, seed=args.seed + rank)
+    B, T, K, C = w.B, w.T, w.K, w.C
+    sumL, terms_pass, bytes_path = algorithmic(w)
+    stream = torch.cuda.current_stream(dev)
+
+    x = torch.from_numpy(w.x).to(dev)
+    A = torch.from_numpy(w.A).to(dev)
+    D = torch.from_numpy(w.D).to(dev)
+    lens = torch.from_numpy(w.lengths).to(dev)
+    ws = sc.new_workspace(B, T, K, C, sc.WS_TRAIN, args.ckpt, device=dev)
+    S = torch.empty((B, T + 1, C), dtype=torch.float64, device=dev)
+    nu = torch.empty((B, C), dtype=torch.float64, device=dev)
+    logZ = torch.empty(B, dtype=torch.float64, device=dev)
+    dX = torch.empty((B, T, C), dtype=torch.float32, device=dev)
+    dA = torch.empty((C, C), dtype=torch.float64, device=dev)
+    dD = torch.empty((K, C), dtype=torch.float64, device=dev)
+    flush = torch.empty(256 * 2**20 // 4, dtype=torch.float32, device=dev)
+
+    # per-kernel events (recorded by the library around each launch)
+    n_ev = 2 * len(KERNEL_NAMES)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    for e in evs:
+        e.record(stream)
+    handles = (ctypes_void_p_array(len(evs)))(*[e.cuda_event for e in evs])
+    lib = _lib.load()
+
+    def step(profile=False):
+        if profile:
+            lib.semicrf_set_profile_events(handles, 6)
+        sc.prefix_scan(x, lens, ws=ws, S=S, nu=nu)
+        if profile:
+            lib.semicrf_set_profile_events(ctypes_offset(handles, 6), 2)
+        sc.forward(S, A, D, lens, ws=ws, ckpt_interval=args.ckpt, logZ=logZ)
+        if profile:
+            lib.semicrf_set_profile_events(ctypes_offset(handles, 8), 8)
+        sc.backward(S, A, D, lens, ws, ckpt_interval=args.ckpt, dX=dX, dA=dA, dD=dD)
+        if profile:
+            lib.semicrf_set_profile_events(None, 0)
+        if world > 1:
+            dist.all_reduce(dA)
+            dist.all_reduce(dD)
+
+    sc.clear_device_status(ws)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = sc.device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {sc.status_string(status)}")
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_ms, kern_ms = [], {n: 0.0 for n in KERNEL_NAMES}
+    wall0 = time.perf_counter()
+    for _ in range(args.steps):
+        flush.zero_()                       # L2 flush between timed steps (not timed)
+        t_start.record(stream)
+        step(profile=True)
+        t_end.record(stream)
+        t_end.synchronize()
+        step_ms.append(t_start.elapsed_time(t_end))
+        for i, n in enumerate(KERNEL_NAMES):
+            kern_ms[n] += evs[2 * i].elapsed_time(evs[2 * i + 1])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    clk = clocks.stop() if rank == 0 else None
+    status = sc.device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status after timing: {sc.status_string(status)}")
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hx = torch.from_numpy(w.x).pin_memory()
+        hA = torch.from_numpy(w.A).pin_memory()
+        hD = torch.from_numpy(w.D).pin_memory()
+        hl = torch.from_numpy(w.lengths).pin_memory()
+        h_logZ = torch.empty(B, dtype=torch.float64).pin_memory()
+        h_dA = torch.empty((C, C), dtype=torch.float64).pin_memory()
+        h_dD = torch.empty((K, C), dtype=torch.float64).pin_memory()
+        h2d = hx.numel() * 4 + hA.numel() * 4 + hD.numel() * 4 + hl.numel() * 4
+        d2h = h_logZ.numel() * 8 + h_dA.numel() * 8 + h_dD.numel() * 8
+
+        def e2e_step():
+            x.copy_(hx, non_blocking=True)
+            A.copy_(hA, non_blocking=True)
+            D.copy_(hD, non_blocking=True)
+            lens.copy_(hl, non_blocking=True)
+            step()
+            h_logZ.copy_(logZ, non_blocking=True)
+            h_dA.copy_(dA, non_blocking=True)
+            h_dD.copy_(dD, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        e_ms = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            t_start.record(stream)
+            e2e_step()
+            t_end.record(stream)
+            t_end.synchronize()
+            e_ms += t_start.elapsed_time(t_end)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * w.updates * args.steps / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return None
+
+    # ---- roofline of the dominant kernel
+    peaks = measured_peaks() or {}
+    sm_max = float(peaks.get("sm_max_mhz", SM_MAX_MHZ_FALLBACK))
+    fp64_peak_tflops = N_SM * FP64_FMA_PER_SM_CLK * 2 * sm_max * 1e6 / 1e12
+    dom = max(kern_ms, key=kern_ms.get)
+    per_launch_ms = kern_ms[dom] / args.steps
+    work_flop = {"fwd_kernel": 2 * terms_pass, "bwd_kernel": 2 * terms_pass,
+                 "fwd_recompute": 2 * terms_pass}
+    if dom in work_flop:
+        achieved = work_flop[dom] / (per_launch_ms / 1e3) / 1e12
+        roof = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": fp64_peak_tflops,
+                "unit": "TFLOP/s", "frac": achieved / fp64_peak_tflops, "traffic": None,
+                "peak_source": f"derived: {N_SM} SMs x {FP64_FMA_PER_SM_CLK} FP64 FMA/clk x 2 x {sm_max:.0f} MHz",
+                "work": "2 flop per (log-sum-exp, +) term: sum_b L_b (K*C + C*C) terms per launch"}
+    else:
+        hbm = float(peaks.get("hbm_gbs", HBM_FALLBACK_GBS))
+        nbytes = 4 * B * T * C + 8 * B * (T + 1) * C
+        achieved = nbytes / (per_launch_ms / 1e3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": None}
+    # the roofline as the workload defines it: slower of HBM bytes and MUFU exps
+    hbm = float(peaks.get("hbm_gbs", HBM_FALLBACK_GBS))
+    t_hbm = bytes_path / (hbm * 1e9)
+    t_sfu = 2 * terms_pass / (N_SM * MUFU_PER_SM_CLK * sm_max * 1e6)
+    t_fp64 = 2 * terms_pass / (N_SM * FP64_FMA_PER_SM_CLK * sm_max * 1e6)
+    ms = total_ms / args.steps
+    value = world * w.updates * args.steps / (total_ms / 1e3)
+    kern_share = {n: round(kern_ms[n] / max(1e-9, sum(kern_ms.values())), 4) for n in KERNEL_NAMES}
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.config, "B": B, "T": T, "K": K, "C": C,
+                   "ckpt_interval": args.ckpt or int(math.ceil(math.sqrt(T))), "seed": args.seed,
+                   "sum_lengths": sumL, "valid_updates_per_s": world * w.valid_updates * args.steps / (total_ms / 1e3),
+                   "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"dp{world}"},
+        "roofline": roof,
+        "roofline_workload": {"t_hbm_ms": t_hbm * 1e3, "t_sfu_ms": t_sfu * 1e3, "t_fp64_ms": t_fp64 * 1e3,
+                              "t_step_ms": ms, "frac_sfu": t_sfu * 1e3 / ms, "frac_fp64": t_fp64 * 1e3 / ms},
+        "kernel_ms_per_step": {n: kern_ms[n] / args.steps for n in KERNEL_NAMES},
+        "kernel_share": kern_share,
+        "gpu_launches": 8 * args.steps,
+        "e2e": e2e,
+        "clocks": clk,
+        "wall_s": wall,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = oracle_sample(w, budget_s=args.cpu_budget)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return out
+
+
+def ctypes_void_p_array(n):
+    import ctypes
+    return ctypes.c_void_p * n
+
+
+def ctypes_offset(arr, k):
+    import ctypes
+    return ctypes.cast(ctypes.byref(arr, k * ctypes.sizeof(ctypes.c_void_p)), ctypes.POINTER(ctypes.c_void_p))
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    w = wl.make_workload(args.config, seed=args.seed)
+    budget = max(0.5, args.cpu_budget / max(1, args.steps))
+    for _ in range(args.warmup if args.warmup < 2 else 1):
+        oracle_sample(w, budget_s=0.01)
+    vals = []
+    t0 = time.perf_counter()
+    info = None
+    for _ in range(args.steps):
+        info = oracle_sample(w, budget_s=budget)
+        vals.append(info["value"])
+    el = time.perf_counter() - t0
+    value = statistics.median(vals)
+    cb = dict(info)
+    cb["value"] = value
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": args.config, "B": w.B, "T": w.T, "K": w.K, "C": w.C, "seed": args.seed,
+                   "parallelism": "cpu"},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="ner", choices=[k for k in wl.CONFIGS if k != "tiny10"])
+    ap.add_argument("--ckpt", type=int, default=0, help="checkpoint interval (0: ceil(sqrt(T)))")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    out = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

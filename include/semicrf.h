@@ -1,0 +1,164 @@
+/*
+ * semicrf.h -- C ABI of libsemicrf.so: exact semi-CRF streaming forward-backward
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The operation is the semi-Markov CRF of "Streaming Structured Inference with
+ * Flash-SemiCRF" (abstract; technical summary sections 1-2): segments [s, s+d)
+ * with label c score S[s+d,c] - S[s,c] + D[d-1,c], consecutive segments add
+ * A[c',c], S is the prefix sum of zero-centred emissions (section 2.A, 2.C), and
+ * the library returns log Z, its exact gradients (section 2.C: checkpointed
+ * streaming forward-backward with local recompute) and the Viterbi segmentation.
+ *
+ * Shapes (all row-major, contiguous, last index fastest):
+ *   x          float32 [B, T, C]    emissions; positions t >= L_b are never read
+ *   lengths    int32   [B]          L_b in [1, T]  (checked on the device)
+ *   S          float64 [B, T+1, C]  prefix sums of centred emissions
+ *   nu         float64 [B, C]       centring baseline (mean over t < L_b)
+ *   A          float32 [C, C]       transition score, A[from, to]
+ *   D          float32 [K, C]       duration bias, row d-1 for duration d
+ *   logZ       float64 [B]
+ *   grad_logZ  float64 [B]          upstream weights g_b, or NULL for all ones
+ *   dX         float32 [B, T, C]    g_b * dlogZ_b/dx (through S and nu); 0 for t >= L_b
+ *   dA         float64 [C, C]       sum_b g_b dlogZ_b/dA
+ *   dD         float64 [K, C]       sum_b g_b dlogZ_b/dD
+ *   score      float64 [B]          Viterbi score
+ *   labels     int32   [B, T]       Viterbi label per position, -1 for t >= L_b
+ *   seg_start  uint8   [B, T]       1 where a Viterbi segment begins, else 0
+ *
+ * Ownership and execution: every data pointer is caller-owned DEVICE memory
+ * (except where a function says otherwise).  The library allocates nothing and
+ * frees nothing.  Every call is asynchronous on the caller's CUDA stream, passed
+ * as an opaque pointer (a cudaStream_t; NULL is the legacy default stream), and
+ * returns after launching.  Only semicrf_get_device_status synchronises.
+ *
+ * Workspace: the caller provides `ws` of at least semicrf_workspace_bytes(dims,
+ * what) bytes, 256-byte aligned.  The same workspace must be passed unchanged
+ * from semicrf_forward to semicrf_backward (it holds the checkpoints and the
+ * log-normaliser).  semicrf_prefix_scan also uses it (scratch for chunk sums).
+ *
+ * Errors: argument checks happen on the host before any launch and return a
+ * status; nothing is launched then.  Device-side findings (a length outside
+ * [1, T], a non-finite log Z) are recorded in the workspace's status word and
+ * read back by semicrf_get_device_status.  Outputs of a call that found an
+ * error are unspecified.
+ */
+#ifndef SEMICRF_H
+#define SEMICRF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SEMICRF_OK = 0,
+    SEMICRF_ERR_INVALID_ARG = 1,        /* null pointer, non-positive size, bad flag   */
+    SEMICRF_ERR_UNSUPPORTED_SHAPE = 2,  /* K or C beyond the compiled limits           */
+    SEMICRF_ERR_WORKSPACE_TOO_SMALL = 3,
+    SEMICRF_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed        */
+    SEMICRF_ERR_DEVICE_TIMEOUT = 5,     /* a bounded device-side wait expired          */
+    SEMICRF_ERR_DEVICE_RANGE = 6,       /* device saw a non-finite normaliser          */
+    SEMICRF_ERR_INVALID_LENGTH = 7      /* device saw a length outside [1, T]          */
+} semicrf_status;
+
+/* Problem dimensions.  ckpt_interval is the checkpoint spacing Delta in positions
+ * (0 selects ceil(sqrt(T))); results do not depend on it. */
+typedef struct {
+    int32_t B, T, K, C;
+    int32_t ckpt_interval;
+} semicrf_dims;
+
+/* what: which calls the workspace serves (a TRAIN or VITERBI workspace also
+ * serves prefix_scan) */
+#define SEMICRF_WS_TRAIN 0   /* prefix_scan + forward + backward */
+#define SEMICRF_WS_VITERBI 1 /* prefix_scan + viterbi            */
+#define SEMICRF_WS_SCAN 2    /* prefix_scan only                 */
+
+/* Compiled limits (SEMICRF_ERR_UNSUPPORTED_SHAPE beyond them). */
+#define SEMICRF_MAX_C 256
+#define SEMICRF_MAX_K 4096
+
+/*
+ * Bytes of device workspace needed for `what` at these dims; 0 if the dims are
+ * invalid or unsupported (semicrf_check_dims says which).
+ */
+size_t semicrf_workspace_bytes(const semicrf_dims *dims, int32_t what);
+
+/* Host check of dims alone (no CUDA calls). */
+semicrf_status semicrf_check_dims(const semicrf_dims *dims);
+
+/*
+ * Centring and prefix scan (technical summary 2.A and 2.C):
+ *   nu[b,c]    = (1/L_b) sum_{t<L_b} x[b,t,c]
+ *   S[b,0,c]   = 0,  S[b,t+1,c] = S[b,t,c] + x[b,t,c] - nu[b,c]  (t < L_b)
+ *   S[b,t,c]   = S[b,L_b,c] for t > L_b
+ * Accumulates in float64; x rows t >= L_b are not read.
+ */
+semicrf_status semicrf_prefix_scan(const semicrf_dims *dims, const float *x,
+                                   const int32_t *lengths, double *S, double *nu,
+                                   void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Streaming forward (abstract: prefix-sum lookup instead of an edge tensor;
+ * technical summary 2.B-2.C: O(K*C) ring of forward messages, normalised
+ * checkpoints every ckpt_interval positions).  Writes logZ[b] and keeps the
+ * checkpoints and log-normaliser in ws for semicrf_backward.
+ */
+semicrf_status semicrf_forward(const semicrf_dims *dims, const double *S, const float *A,
+                               const float *D, const int32_t *lengths, double *logZ,
+                               void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Backward (technical summary 2.C: recompute the forward messages inside each
+ * checkpoint segment, stream the backward messages through a K*C ring, form the
+ * segment and transition marginals).  Overwrites dX, dA, dD with the exact
+ * gradients of sum_b g_b logZ_b, where g = grad_logZ (NULL: ones).  ws must be the
+ * workspace the matching semicrf_forward call used.
+ */
+semicrf_status semicrf_backward(const semicrf_dims *dims, const double *S, const float *A,
+                                const float *D, const int32_t *lengths,
+                                const double *grad_logZ, void *ws, size_t ws_bytes,
+                                float *dX, double *dA, double *dD, void *stream);
+
+/*
+ * Viterbi: the forward recursion in (max, +), float64.  Ties pick the smallest
+ * duration, then the smallest previous label; the final label is the smallest
+ * reaching the maximum.  (The pages do not describe decoding; this follows the
+ * same segment score.)
+ */
+semicrf_status semicrf_viterbi(const semicrf_dims *dims, const double *S, const float *A,
+                               const float *D, const int32_t *lengths, double *score,
+                               int32_t *labels, uint8_t *seg_start, void *ws,
+                               size_t ws_bytes, void *stream);
+
+/* Zero the device status word in ws (asynchronous on stream). */
+semicrf_status semicrf_clear_device_status(void *ws, void *stream);
+
+/*
+ * Synchronise `stream`, read the device status word from ws and return it
+ * (SEMICRF_OK when no device-side error was recorded).
+ */
+semicrf_status semicrf_get_device_status(const void *ws, void *stream);
+
+/* Static, human-readable name of a status. */
+const char *semicrf_status_string(semicrf_status s);
+
+/* Kernel launches issued by the most recent successful call on this thread. */
+int32_t semicrf_last_launch_count(void);
+
+/*
+ * Per-kernel timing for profilers and benchmarks.  `events` points to n
+ * caller-created cudaEvent_t handles (host array; the library keeps the pointer,
+ * so it must stay valid while set).  While set, each API call on this thread
+ * records events[2i] just before and events[2i+1] just after its i-th kernel
+ * launch (i < n/2), on the call's stream.  Pass NULL, 0 to stop.
+ */
+semicrf_status semicrf_set_profile_events(void *const *events, int32_t n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEMICRF_H */

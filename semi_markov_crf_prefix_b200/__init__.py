@@ -1,0 +1,169 @@
+"""B200-native exact semi-CRF: prefix-sum segment scores, streaming forward-
+backward with checkpoints, exact gradients, Viterbi.
+
+Thin binding over ``libsemicrf.so`` (C ABI in ``include/semicrf.h``): this module
+only marshals torch CUDA tensors into the library's calls on the current CUDA
+stream.  Every step of the computation runs in the library's kernels; there is
+no CPU or PyTorch fallback.
+
+Layout (row-major): x float32 [B,T,C]; A float32 [C,C] (from, to); D float32
+[K,C] (row d-1); lengths int32 [B]; S float64 [B,T+1,C]; logZ float64 [B];
+dX float32 [B,T,C]; dA float64 [C,C]; dD float64 [K,C].
+"""
+from __future__ import annotations
+
+import ctypes
+
+from . import _lib
+from ._lib import (MAX_C, MAX_K, WS_SCAN, WS_TRAIN, WS_VITERBI, SemiCRFError, dims,
+                   status_string)
+
+__all__ = ["workspace_bytes", "new_workspace", "prefix_scan", "forward", "backward", "viterbi",
+           "logz_and_grads", "device_status", "clear_device_status", "last_launch_count",
+           "SemiCRFError", "status_string", "MAX_C", "MAX_K", "WS_TRAIN", "WS_VITERBI", "WS_SCAN",
+           "load_library"]
+
+
+def load_library():
+    return _lib.load()
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(device=None):
+    torch = _torch()
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t, dtype, shape, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def workspace_bytes(B, T, K, C, what=WS_TRAIN, ckpt_interval=0) -> int:
+    d = dims(B, T, K, C, ckpt_interval)
+    n = _lib.load().semicrf_workspace_bytes(ctypes.byref(d), int(what))
+    if n == 0:
+        _lib.check(_lib.load().semicrf_check_dims(ctypes.byref(d)), "workspace_bytes")
+    return int(n)
+
+
+def new_workspace(B, T, K, C, what=WS_TRAIN, ckpt_interval=0, device="cuda"):
+    """A device workspace (uint8 tensor, 256-byte aligned by the caching allocator)."""
+    torch = _torch()
+    n = workspace_bytes(B, T, K, C, what, ckpt_interval)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def prefix_scan(x, lengths, ws=None, S=None, nu=None):
+    """nu [B,C] and S [B,T+1,C] (float64) from x [B,T,C] float32."""
+    torch = _torch()
+    B, T, C = x.shape
+    _need(x, torch.float32, (B, T, C), "x")
+    _need(lengths, torch.int32, (B,), "lengths")
+    if ws is None:
+        ws = new_workspace(B, T, 1, C, WS_SCAN, device=x.device)
+    S = torch.empty((B, T + 1, C), dtype=torch.float64, device=x.device) if S is None else S
+    nu = torch.empty((B, C), dtype=torch.float64, device=x.device) if nu is None else nu
+    d = dims(B, T, 1, C)
+    _lib.check(_lib.load().semicrf_prefix_scan(ctypes.byref(d), _ptr(x), _ptr(lengths), _ptr(S), _ptr(nu),
+                                               _ptr(ws), ws.numel(), _stream(x.device)), "prefix_scan")
+    return S, nu
+
+
+def forward(S, A, D, lengths, ws=None, ckpt_interval=0, logZ=None):
+    """log Z [B] (float64); returns (logZ, ws) -- pass ws unchanged to backward()."""
+    torch = _torch()
+    B, T1, C = S.shape
+    T = T1 - 1
+    K = D.shape[0]
+    _need(S, torch.float64, (B, T + 1, C), "S")
+    _need(A, torch.float32, (C, C), "A")
+    _need(D, torch.float32, (K, C), "D")
+    _need(lengths, torch.int32, (B,), "lengths")
+    if ws is None:
+        ws = new_workspace(B, T, K, C, WS_TRAIN, ckpt_interval, device=S.device)
+    logZ = torch.empty(B, dtype=torch.float64, device=S.device) if logZ is None else logZ
+    d = dims(B, T, K, C, ckpt_interval)
+    _lib.check(_lib.load().semicrf_forward(ctypes.byref(d), _ptr(S), _ptr(A), _ptr(D), _ptr(lengths),
+                                           _ptr(logZ), _ptr(ws), ws.numel(), _stream(S.device)), "forward")
+    return logZ, ws
+
+
+def backward(S, A, D, lengths, ws, grad_logZ=None, ckpt_interval=0, dX=None, dA=None, dD=None):
+    """(dX [B,T,C] float32, dA [C,C] float64, dD [K,C] float64) of sum_b g_b logZ_b."""
+    torch = _torch()
+    B, T1, C = S.shape
+    T = T1 - 1
+    K = D.shape[0]
+    if grad_logZ is not None:
+        _need(grad_logZ, torch.float64, (B,), "grad_logZ")
+    dX = torch.empty((B, T, C), dtype=torch.float32, device=S.device) if dX is None else dX
+    dA = torch.empty((C, C), dtype=torch.float64, device=S.device) if dA is None else dA
+    dD = torch.empty((K, C), dtype=torch.float64, device=S.device) if dD is None else dD
+    d = dims(B, T, K, C, ckpt_interval)
+    _lib.check(_lib.load().semicrf_backward(ctypes.byref(d), _ptr(S), _ptr(A), _ptr(D), _ptr(lengths),
+                                            _ptr(grad_logZ), _ptr(ws), ws.numel(), _ptr(dX), _ptr(dA),
+                                            _ptr(dD), _stream(S.device)), "backward")
+    return dX, dA, dD
+
+
+def viterbi(S, A, D, lengths, ws=None):
+    """(score [B] float64, labels [B,T] int32, seg_start [B,T] uint8)."""
+    torch = _torch()
+    B, T1, C = S.shape
+    T = T1 - 1
+    K = D.shape[0]
+    _need(S, torch.float64, (B, T + 1, C), "S")
+    _need(A, torch.float32, (C, C), "A")
+    _need(D, torch.float32, (K, C), "D")
+    _need(lengths, torch.int32, (B,), "lengths")
+    if ws is None:
+        ws = new_workspace(B, T, K, C, WS_VITERBI, device=S.device)
+    score = torch.empty(B, dtype=torch.float64, device=S.device)
+    labels = torch.empty((B, T), dtype=torch.int32, device=S.device)
+    seg = torch.empty((B, T), dtype=torch.uint8, device=S.device)
+    d = dims(B, T, K, C)
+    _lib.check(_lib.load().semicrf_viterbi(ctypes.byref(d), _ptr(S), _ptr(A), _ptr(D), _ptr(lengths),
+                                           _ptr(score), _ptr(labels), _ptr(seg), _ptr(ws), ws.numel(),
+                                           _stream(S.device)), "viterbi")
+    return score, labels, seg
+
+
+def logz_and_grads(x, A, D, lengths, grad_logZ=None, ckpt_interval=0, ws=None):
+    """prefix_scan + forward + backward: (logZ, dX, dA, dD, ws)."""
+    B, T, C = x.shape
+    K = D.shape[0]
+    if ws is None:
+        ws = new_workspace(B, T, K, C, WS_TRAIN, ckpt_interval, device=x.device)
+    S, _ = prefix_scan(x, lengths, ws=ws)
+    logZ, ws = forward(S, A, D, lengths, ws=ws, ckpt_interval=ckpt_interval)
+    dX, dA, dD = backward(S, A, D, lengths, ws, grad_logZ=grad_logZ, ckpt_interval=ckpt_interval)
+    return logZ, dX, dA, dD, ws
+
+
+def clear_device_status(ws):
+    _lib.check(_lib.load().semicrf_clear_device_status(_ptr(ws), _stream(ws.device)), "clear_device_status")
+
+
+def device_status(ws) -> int:
+    """Synchronise the current stream and return the workspace's device status code."""
+    return int(_lib.load().semicrf_get_device_status(_ptr(ws), _stream(ws.device)))
+
+
+def last_launch_count() -> int:
+    return int(_lib.load().semicrf_last_launch_count())

@@ -1,0 +1,356 @@
+// semicrf_api.cu -- the extern "C" boundary of libsemicrf.so: argument checks,
+// launch planning, workspace layout and kernel launches on the caller's stream.
+// No allocation, no synchronisation (except semicrf_get_device_status).
+#include <math.h>
+#include <string.h>
+
+#include "semicrf_internal.h"
+
+namespace semicrf {
+
+namespace {
+thread_local int g_last_launches = 0;
+thread_local void *const *g_prof_events = nullptr;
+thread_local int g_prof_n = 0;
+thread_local int g_prof_i = 0;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int round_up_pow2(int v, int lo)
+{
+    int x = lo;
+    while (x < v) x <<= 1;
+    return x;
+}
+}  // namespace
+
+void prof_reset() { g_prof_i = 0; }
+
+void prof_before(cudaStream_t st)
+{
+    if (g_prof_events && 2 * g_prof_i + 1 < g_prof_n)
+        cudaEventRecord(static_cast<cudaEvent_t>(g_prof_events[2 * g_prof_i]), st);
+}
+
+void prof_after(cudaStream_t st)
+{
+    if (g_prof_events && 2 * g_prof_i + 1 < g_prof_n)
+        cudaEventRecord(static_cast<cudaEvent_t>(g_prof_events[2 * g_prof_i + 1]), st);
+    ++g_prof_i;
+}
+
+int default_delta(int T)
+{
+    int d = (int)ceil(sqrt((double)T));
+    return d < 1 ? 1 : d;
+}
+
+// Smallest cluster (G CTAs, labels split evenly) whose per-CTA shared memory and
+// per-thread register tiles fit, preferring <= 12288 duration+transition terms
+// per CTA per step so that a step stays short.
+Plan make_plan(int K, int C)
+{
+    Plan best;
+    const int Gs[] = {1, 2, 4, 8, 16};
+    for (int gi = 0; gi < 5; ++gi) {
+        const int G = Gs[gi];
+        if (G > C) break;
+        Plan p;
+        p.G = G;
+        p.Cg = (C + G - 1) / G;
+        if ((G - 1) * p.Cg >= C) continue;   // every CTA must own at least one label
+        const long work = (long)(K + C) * p.Cg;
+        int nt = (int)align_up((size_t)((work + 15) / 16), 32);
+        if (nt < 32) nt = 32;
+        if (nt > kMaxThreads) nt = kMaxThreads;
+        if (nt < p.Cg) nt = (int)align_up((size_t)p.Cg, 32);
+        if (nt > kMaxThreads) continue;
+        p.NT = nt;
+        p.JL = nt / p.Cg;
+        p.DPT = round_up_pow2((K + p.JL - 1) / p.JL, 2);
+        p.CPT = round_up_pow2((C + p.JL - 1) / p.JL, 2);
+        if (p.DPT > 32 || p.CPT > 16) continue;
+        const size_t ring = (size_t)K * p.Cg * 8;
+        const size_t common = 2 * (size_t)C * 8 + (size_t)nt * 8 + 64;
+        p.smem_fwd = ring + common + (size_t)p.Cg * 4 + 16;
+        p.smem_bwd = 2 * ring + common + (size_t)p.Cg * 20 + 16;
+        p.smem_vit = 2 * ring + common + (size_t)nt * 4;
+        if (p.smem_bwd > kSmemBudget || p.smem_vit > kSmemBudget) continue;
+        best = p;
+        if (work <= 12288) break;
+    }
+    return best;
+}
+
+bool make_layout(const semicrf_dims &d, int what, const Plan &p, Layout *out)
+{
+    (void)p;
+    Layout L;
+    const size_t B = d.B, T = d.T, K = d.K, C = d.C;
+    L.delta = d.ckpt_interval > 0 ? d.ckpt_interval : default_delta(d.T);
+    if (L.delta > d.T) L.delta = d.T;
+    L.J = (d.T + L.delta - 1) / L.delta;
+    int nch = (296 + d.B - 1) / d.B;
+    int maxch = (d.T + 63) / 64;
+    if (nch > maxch) nch = maxch;
+    if (nch < 1) nch = 1;
+    L.NCH = nch;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    L.status = take(16);
+    L.scan = take(B * L.NCH * C * 8);
+    if (what == SEMICRF_WS_TRAIN) {
+        L.logz = take(B * sizeof(LogZState));
+        L.ckpt_stride = align_up(K * C * 8 + (C + 1) * 4, 256);
+        L.ckpt = take(B * (size_t)L.J * L.ckpt_stride);
+        L.aU = take(B * (T + 1) * C * 8);
+        L.aA = take(B * (T + 1) * C * 8);
+        L.aR = take(B * (T + 1) * C * 4);
+        L.aK = take(B * (T + 1) * 4);
+        L.accD = take(B * K * C * 8);
+        L.accA = take(B * C * C * 8);
+        L.musum = take(B * C * 8);
+        L.mures = take(B * C * 8);
+        L.logzb = take(B * 8);
+    } else if (what == SEMICRF_WS_VITERBI) {
+        L.bd = take(B * (T + 1) * C * 2);
+        L.bc = take(B * (T + 1) * C * 2);
+        L.vfin = take(B * 4);
+    } else if (what != SEMICRF_WS_SCAN) {
+        return false;
+    }
+    L.total = off;
+    *out = L;
+    return true;
+}
+
+}  // namespace semicrf
+
+using namespace semicrf;
+
+namespace {
+
+semicrf_status check_dims_impl(const semicrf_dims *d)
+{
+    if (!d) return SEMICRF_ERR_INVALID_ARG;
+    if (d->B < 1 || d->T < 1 || d->K < 1 || d->C < 1 || d->ckpt_interval < 0)
+        return SEMICRF_ERR_INVALID_ARG;
+    if (d->C > SEMICRF_MAX_C || d->K > SEMICRF_MAX_K) return SEMICRF_ERR_UNSUPPORTED_SHAPE;
+    if ((long long)d->B * (d->T + 1) * d->C > (1LL << 40)) return SEMICRF_ERR_UNSUPPORTED_SHAPE;
+    if (!make_plan(d->K, d->C).ok()) return SEMICRF_ERR_UNSUPPORTED_SHAPE;
+    return SEMICRF_OK;
+}
+
+semicrf_status prepare(const semicrf_dims *d, int what, void *ws, size_t ws_bytes, Plan *p,
+                       Layout *lay)
+{
+    prof_reset();
+    semicrf_status s = check_dims_impl(d);
+    if (s != SEMICRF_OK) return s;
+    if (!ws) return SEMICRF_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return SEMICRF_ERR_INVALID_ARG;
+    *p = make_plan(d->K, d->C);
+    if (!make_layout(*d, what, *p, lay)) return SEMICRF_ERR_INVALID_ARG;
+    if (ws_bytes < lay->total) return SEMICRF_ERR_WORKSPACE_TOO_SMALL;
+    return SEMICRF_OK;
+}
+
+template <typename T>
+T *at(void *ws, size_t off)
+{
+    return reinterpret_cast<T *>(static_cast<unsigned char *>(ws) + off);
+}
+
+semicrf_status finish(cudaError_t e, int launches)
+{
+    if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
+    g_last_launches = launches;
+    return SEMICRF_OK;
+}
+
+FbArgs fb_args(const semicrf_dims *d, const Layout &lay, void *ws)
+{
+    FbArgs a;
+    memset(&a, 0, sizeof(a));
+    a.B = d->B;
+    a.T = d->T;
+    a.K = d->K;
+    a.C = d->C;
+    a.delta = lay.delta;
+    a.J = lay.J;
+    a.lz = at<LogZState>(ws, lay.logz);
+    a.ckpt = at<unsigned char>(ws, lay.ckpt);
+    a.ckpt_stride = lay.ckpt_stride;
+    a.aU = at<double>(ws, lay.aU);
+    a.aA = at<double>(ws, lay.aA);
+    a.aR = at<int32_t>(ws, lay.aR);
+    a.aK = at<int32_t>(ws, lay.aK);
+    a.accD = at<double>(ws, lay.accD);
+    a.accA = at<double>(ws, lay.accA);
+    a.musum = at<double>(ws, lay.musum);
+    a.mures = at<double>(ws, lay.mures);
+    a.logzb = at<double>(ws, lay.logzb);
+    a.status = at<int32_t>(ws, lay.status);
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+semicrf_status semicrf_check_dims(const semicrf_dims *dims) { return check_dims_impl(dims); }
+
+size_t semicrf_workspace_bytes(const semicrf_dims *dims, int32_t what)
+{
+    if (check_dims_impl(dims) != SEMICRF_OK) return 0;
+    Plan p = make_plan(dims->K, dims->C);
+    Layout lay;
+    if (!make_layout(*dims, what, p, &lay)) return 0;
+    return lay.total;
+}
+
+semicrf_status semicrf_prefix_scan(const semicrf_dims *dims, const float *x, const int32_t *lengths,
+                                   double *S, double *nu, void *ws, size_t ws_bytes, void *stream)
+{
+    Plan p;
+    Layout lay;
+    // status and scan regions sit at the same offsets in every workspace kind
+    semicrf_status s = prepare(dims, SEMICRF_WS_SCAN, ws, ws_bytes, &p, &lay);
+    if (s != SEMICRF_OK) return s;
+    if (!x || !lengths || !S || !nu) return SEMICRF_ERR_INVALID_ARG;
+    ScanArgs a;
+    a.B = dims->B;
+    a.T = dims->T;
+    a.C = dims->C;
+    a.NCH = lay.NCH;
+    a.x = x;
+    a.lengths = lengths;
+    a.S = S;
+    a.nu = nu;
+    a.part = at<double>(ws, lay.scan);
+    a.status = at<int32_t>(ws, lay.status);
+    int n = 0;
+    cudaError_t e = launch_prefix_scan(a, static_cast<cudaStream_t>(stream), &n);
+    return finish(e, n);
+}
+
+semicrf_status semicrf_forward(const semicrf_dims *dims, const double *S, const float *A, const float *D,
+                               const int32_t *lengths, double *logZ, void *ws, size_t ws_bytes,
+                               void *stream)
+{
+    Plan p;
+    Layout lay;
+    semicrf_status s = prepare(dims, SEMICRF_WS_TRAIN, ws, ws_bytes, &p, &lay);
+    if (s != SEMICRF_OK) return s;
+    if (!S || !A || !D || !lengths || !logZ) return SEMICRF_ERR_INVALID_ARG;
+    FbArgs a = fb_args(dims, lay, ws);
+    a.S = S;
+    a.A = A;
+    a.D = D;
+    a.lengths = lengths;
+    a.logZ = logZ;
+    int n = 0;
+    cudaError_t e = launch_forward(p, a, static_cast<cudaStream_t>(stream), &n);
+    return finish(e, n);
+}
+
+semicrf_status semicrf_backward(const semicrf_dims *dims, const double *S, const float *A, const float *D,
+                                const int32_t *lengths, const double *grad_logZ, void *ws,
+                                size_t ws_bytes, float *dX, double *dA, double *dD, void *stream)
+{
+    Plan p;
+    Layout lay;
+    semicrf_status s = prepare(dims, SEMICRF_WS_TRAIN, ws, ws_bytes, &p, &lay);
+    if (s != SEMICRF_OK) return s;
+    if (!S || !A || !D || !lengths || !dX || !dA || !dD) return SEMICRF_ERR_INVALID_ARG;
+    FbArgs a = fb_args(dims, lay, ws);
+    a.S = S;
+    a.A = A;
+    a.D = D;
+    a.lengths = lengths;
+    a.grad = grad_logZ;
+    a.dX = dX;
+    a.dA = dA;
+    a.dD = dD;
+    int n = 0;
+    cudaError_t e = launch_backward(p, a, static_cast<cudaStream_t>(stream), &n);
+    return finish(e, n);
+}
+
+semicrf_status semicrf_viterbi(const semicrf_dims *dims, const double *S, const float *A, const float *D,
+                               const int32_t *lengths, double *score, int32_t *labels,
+                               uint8_t *seg_start, void *ws, size_t ws_bytes, void *stream)
+{
+    Plan p;
+    Layout lay;
+    semicrf_status s = prepare(dims, SEMICRF_WS_VITERBI, ws, ws_bytes, &p, &lay);
+    if (s != SEMICRF_OK) return s;
+    if (!S || !A || !D || !lengths || !score || !labels || !seg_start) return SEMICRF_ERR_INVALID_ARG;
+    VitArgs a;
+    a.B = dims->B;
+    a.T = dims->T;
+    a.K = dims->K;
+    a.C = dims->C;
+    a.S = S;
+    a.A = A;
+    a.D = D;
+    a.lengths = lengths;
+    a.score = score;
+    a.labels = labels;
+    a.seg_start = seg_start;
+    a.bd = at<uint16_t>(ws, lay.bd);
+    a.bc = at<uint16_t>(ws, lay.bc);
+    a.vfin = at<int32_t>(ws, lay.vfin);
+    a.status = at<int32_t>(ws, lay.status);
+    int n = 0;
+    cudaError_t e = launch_viterbi(p, a, static_cast<cudaStream_t>(stream), &n);
+    return finish(e, n);
+}
+
+semicrf_status semicrf_clear_device_status(void *ws, void *stream)
+{
+    if (!ws) return SEMICRF_ERR_INVALID_ARG;
+    cudaError_t e = cudaMemsetAsync(ws, 0, 16, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SEMICRF_OK : SEMICRF_ERR_CUDA;
+}
+
+semicrf_status semicrf_get_device_status(const void *ws, void *stream)
+{
+    if (!ws) return SEMICRF_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SEMICRF_ERR_CUDA;
+    int32_t h = 0;
+    if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return SEMICRF_ERR_CUDA;
+    return static_cast<semicrf_status>(h);
+}
+
+const char *semicrf_status_string(semicrf_status s)
+{
+    switch (s) {
+    case SEMICRF_OK: return "ok";
+    case SEMICRF_ERR_INVALID_ARG: return "invalid argument";
+    case SEMICRF_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case SEMICRF_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case SEMICRF_ERR_CUDA: return "CUDA error";
+    case SEMICRF_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case SEMICRF_ERR_DEVICE_RANGE: return "non-finite value on device";
+    case SEMICRF_ERR_INVALID_LENGTH: return "sequence length outside [1, T]";
+    }
+    return "unknown status";
+}
+
+int32_t semicrf_last_launch_count(void) { return g_last_launches; }
+
+semicrf_status semicrf_set_profile_events(void *const *events, int32_t n)
+{
+    if (n < 0 || (n > 0 && !events)) return SEMICRF_ERR_INVALID_ARG;
+    g_prof_events = n > 0 ? events : nullptr;
+    g_prof_n = n;
+    g_prof_i = 0;
+    return SEMICRF_OK;
+}
+
+}  // extern "C"

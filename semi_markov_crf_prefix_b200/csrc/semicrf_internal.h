@@ -1,0 +1,114 @@
+// semicrf_internal.h -- host-side launch plan, workspace layout and launcher
+// declarations shared by the translation units of libsemicrf.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "semicrf.h"
+
+namespace semicrf {
+
+// Ring columns are rebased (scaled by an exact power of two) when the weighted
+// column sum leaves [2^-kRebaseBits, 2^kRebaseBits].
+constexpr int kRebaseBits = 256;
+constexpr int kMaxThreads = 512;
+constexpr size_t kSmemBudget = 220 * 1024;
+
+// Per-sequence log-normaliser of the forward pass: log Z = ln2 * k + logn.
+struct LogZState {
+    double logn;
+    int32_t k;
+    int32_t pad;
+};
+
+// How one sequence is spread over a thread-block cluster.  CTA g of the cluster
+// owns labels [g*Cg, min(C, (g+1)*Cg)).  Inside a CTA thread tid works on label
+// column lc = tid % Cg and lane j = tid / Cg (j < JL); lane j handles durations
+// d = 1 + j + m*JL (m < DPT) and previous/next labels j + m*JL (m < CPT).
+struct Plan {
+    int G = 0, NT = 0, Cg = 0, JL = 0, DPT = 0, CPT = 0;
+    size_t smem_fwd = 0, smem_bwd = 0, smem_vit = 0;
+    bool ok() const { return G > 0; }
+};
+
+// Byte offsets of every region inside the caller's workspace.
+struct Layout {
+    int delta = 0;   // checkpoint interval
+    int J = 0;       // checkpoints per sequence (ceil(T / delta))
+    int NCH = 0;     // prefix-scan chunks per sequence
+    size_t status = 0;      // int32[4]
+    size_t scan = 0;        // double [B][NCH][C]
+    size_t logz = 0;        // LogZState [B]
+    size_t ckpt = 0;        // [B][J] records of ckpt_stride bytes
+    size_t ckpt_stride = 0; // ring double[K*C], r int32[C], k int32
+    size_t aU = 0;          // double [B][T+1][C]   recomputed ring rows
+    size_t aA = 0;          // double [B][T+1][C]   recomputed scaled alpha
+    size_t aR = 0;          // int32  [B][T+1][C]   ring exponent per row
+    size_t aK = 0;          // int32  [B][T+1]      alpha exponent per position
+    size_t accD = 0;        // double [B][K][C]
+    size_t accA = 0;        // double [B][C][C]
+    size_t musum = 0;       // double [B][C]
+    size_t mures = 0;       // double [B][C]
+    size_t logzb = 0;       // double [B]
+    size_t bd = 0;          // uint16 [B][T+1][C]  Viterbi best duration
+    size_t bc = 0;          // uint16 [B][T+1][C]  Viterbi best previous label
+    size_t vfin = 0;        // int32 [B]           Viterbi final label
+    size_t total = 0;
+};
+
+// Optional per-launch event recording (semicrf_set_profile_events).
+void prof_before(cudaStream_t st);
+void prof_after(cudaStream_t st);
+void prof_reset();
+
+Plan make_plan(int K, int C);
+bool make_layout(const semicrf_dims &d, int what, const Plan &p, Layout *out);
+int default_delta(int T);
+
+// Launchers: return cudaSuccess or the launch error.
+struct ScanArgs {
+    int B, T, C, NCH;
+    const float *x;
+    const int32_t *lengths;
+    double *S, *nu, *part;
+    int32_t *status;
+};
+cudaError_t launch_prefix_scan(const ScanArgs &a, cudaStream_t st, int *launches);
+
+struct FbArgs {
+    int B, T, K, C, delta, J;
+    const double *S;
+    const float *A, *D;
+    const int32_t *lengths;
+    const double *grad;
+    double *logZ;
+    LogZState *lz;
+    unsigned char *ckpt;
+    size_t ckpt_stride;
+    double *aU, *aA;
+    int32_t *aR, *aK;
+    double *accD, *accA, *musum, *mures, *logzb;
+    float *dX;
+    double *dA, *dD;
+    int32_t *status;
+};
+cudaError_t launch_forward(const Plan &p, const FbArgs &a, cudaStream_t st, int *launches);
+cudaError_t launch_backward(const Plan &p, const FbArgs &a, cudaStream_t st, int *launches);
+
+struct VitArgs {
+    int B, T, K, C;
+    const double *S;
+    const float *A, *D;
+    const int32_t *lengths;
+    double *score;
+    int32_t *labels;
+    uint8_t *seg_start;
+    uint16_t *bd, *bc;
+    int32_t *vfin;
+    int32_t *status;
+};
+cudaError_t launch_viterbi(const Plan &p, const VitArgs &a, cudaStream_t st, int *launches);
+
+}  // namespace semicrf

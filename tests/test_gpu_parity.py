@@ -1,0 +1,193 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 CPU oracle.
+
+Tolerances (the stated bar): relative error <= 1e-5 on log Z, absolute error
+<= 1e-4 on every gradient entry, bit-exact Viterbi labels and segment starts.
+The path computes in float64, so the tests also hold it to tighter internal
+bounds (marked "precision") that would catch a silent drop to float32.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import bruteforce as bf
+import semicrf_workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+LOGZ_RTOL = 1e-5
+GRAD_ATOL = 1e-4
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def run_gpu(w, ckpt_interval=0, grad=None, x=None, lengths=None):
+    """prefix_scan + forward + backward + viterbi on cuda:0; numpy results."""
+    torch = _torch()
+    import semi_markov_crf_prefix_b200 as sc
+    dev = torch.device("cuda:0")
+    xs = torch.from_numpy(np.ascontiguousarray(w.x if x is None else x)).to(dev)
+    A = torch.from_numpy(w.A).to(dev)
+    D = torch.from_numpy(w.D).to(dev)
+    lens = torch.from_numpy(np.ascontiguousarray(w.lengths if lengths is None else lengths)).to(dev)
+    g = None if grad is None else torch.from_numpy(np.asarray(grad, np.float64)).to(dev)
+    ws = sc.new_workspace(w.B, w.T, w.K, w.C, sc.WS_TRAIN, ckpt_interval, device=dev)
+    sc.clear_device_status(ws)
+    S, nu = sc.prefix_scan(xs, lens, ws=ws)
+    logZ, _ = sc.forward(S, A, D, lens, ws=ws, ckpt_interval=ckpt_interval)
+    dX, dA, dD = sc.backward(S, A, D, lens, ws, grad_logZ=g, ckpt_interval=ckpt_interval)
+    status = sc.device_status(ws)
+    wsv = sc.new_workspace(w.B, w.T, w.K, w.C, sc.WS_VITERBI, device=dev)
+    sc.clear_device_status(wsv)
+    score, labels, seg = sc.viterbi(S, A, D, lens, ws=wsv)
+    vstatus = sc.device_status(wsv)
+    torch.cuda.synchronize()
+    return dict(S=S.cpu().numpy(), nu=nu.cpu().numpy(), logZ=logZ.cpu().numpy(), dX=dX.cpu().numpy(),
+                dA=dA.cpu().numpy(), dD=dD.cpu().numpy(), score=score.cpu().numpy(),
+                labels=labels.cpu().numpy(), seg_start=seg.cpu().numpy(), status=status,
+                vstatus=vstatus)
+
+
+def check_against_oracle(w, g, grad=None, precision=True):
+    o = oracle.factorised(w.x, w.A, w.D, w.lengths, grad_logZ=grad)
+    assert g["status"] == 0 and g["vstatus"] == 0
+    rel = np.abs(g["logZ"] - o["logZ"]) / np.abs(o["logZ"])
+    assert rel.max() <= LOGZ_RTOL, rel.max()
+    for k in ("dX", "dA", "dD"):
+        err = np.abs(g[k] - o[k]).max()
+        assert err <= GRAD_ATOL, (k, err)
+    if precision:
+        assert rel.max() <= 1e-11, ("precision logZ", rel.max())
+        assert np.abs(g["dA"] - o["dA"]).max() <= 1e-8 * max(1.0, np.abs(o["dA"]).max())
+        assert np.abs(g["dD"] - o["dD"]).max() <= 1e-8 * max(1.0, np.abs(o["dD"]).max())
+        assert np.abs(g["dX"] - o["dX"]).max() <= 1e-6
+    s, labels, seg = oracle.viterbi(w.x, w.A, w.D, w.lengths)
+    np.testing.assert_allclose(g["score"], s, rtol=1e-12)
+    assert np.array_equal(g["labels"], labels)
+    assert np.array_equal(g["seg_start"], seg)
+    return o
+
+
+def test_prefix_scan_matches_oracle():
+    w = wl.make_workload("ner")
+    g = run_gpu(w)
+    S, nu = oracle.prefix(w.x, w.lengths)
+    np.testing.assert_allclose(g["nu"], nu, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(g["S"], S, rtol=0, atol=1e-11)
+    for b in range(w.B):
+        L = int(w.lengths[b])
+        assert np.all(g["S"][b, L:] == g["S"][b, L])
+        assert abs(g["S"][b, L]).max() < 1e-10
+
+
+def test_tiny10_against_enumeration():
+    w = wl.make_workload("tiny10")
+    g = run_gpu(w)
+    e = bf.enumerate_batch(w.x, w.A, w.D, w.lengths)
+    np.testing.assert_allclose(g["logZ"], e["logZ"], rtol=1e-12)
+    np.testing.assert_allclose(g["dA"], e["dA"], atol=1e-11)
+    np.testing.assert_allclose(g["dD"], e["dD"], atol=1e-11)
+    np.testing.assert_allclose(g["dX"], e["dX"], atol=1e-6)
+    np.testing.assert_allclose(g["score"], e["score"], rtol=1e-12)
+    assert np.array_equal(g["labels"], e["labels"]) and np.array_equal(g["seg_start"], e["seg_start"])
+
+
+@pytest.mark.parametrize("name", ["tiny", "ner"])
+def test_named_small(name):
+    w = wl.make_workload(name)
+    check_against_oracle(w, run_gpu(w))
+
+
+def test_upstream_weights():
+    w = wl.make_workload("ner")
+    grad = np.random.default_rng(1).normal(size=w.B)
+    check_against_oracle(w, run_gpu(w, grad=grad), grad=grad)
+
+
+def test_speech_full():
+    w = wl.make_workload("speech")
+    check_against_oracle(w, run_gpu(w))
+
+
+def test_genomic_reduced_T():
+    w = wl.make_workload("genomic", T=6000)
+    check_against_oracle(w, run_gpu(w))
+
+
+def test_large_reduced_T():
+    # full K and C (and so the full cluster layout) on a shorter sequence
+    w = wl.make_workload("large", B=2, T=1500)
+    check_against_oracle(w, run_gpu(w))
+
+
+@pytest.mark.parametrize("seed,B,T,K,C", [(0, 3, 37, 5, 3), (1, 5, 100, 1, 7), (2, 2, 70, 70, 2),
+                                           (3, 4, 129, 33, 33), (4, 1, 1, 4, 5), (5, 2, 50, 200, 9),
+                                           (6, 3, 300, 40, 64), (7, 2, 200, 300, 20)])
+def test_random_shapes(seed, B, T, K, C):
+    w = wl.random_small(seed, B, T, K, C, ragged=True)
+    check_against_oracle(w, run_gpu(w))
+
+
+def test_checkpoint_interval_invariance():
+    w = wl.make_workload("ner", B=6)
+    T, K = w.T, w.K
+    ref = run_gpu(w, ckpt_interval=0)
+    for ck in (1, 7, int(math.ceil(math.sqrt(T * K))), T):
+        g = run_gpu(w, ckpt_interval=ck)
+        for k in ("logZ", "dX", "dA", "dD"):
+            assert np.array_equal(g[k], ref[k]), (ck, k)
+
+
+def test_nan_padding_is_never_read():
+    w = wl.make_workload("ner")
+    ref = run_gpu(w)
+    x = w.x.copy()
+    for b in range(w.B):
+        x[b, int(w.lengths[b]):] = np.nan
+    g = run_gpu(w, x=x)
+    for k in ("logZ", "dX", "dA", "dD", "score", "labels", "seg_start"):
+        assert np.array_equal(g[k], ref[k]), k
+
+
+def test_invalid_length_sets_device_status():
+    w = wl.make_workload("tiny")
+    bad = w.lengths.copy()
+    bad[1] = w.T + 1
+    g = run_gpu(w, lengths=bad)
+    assert g["status"] == 7 and g["vstatus"] == 7
+
+
+def test_zero_scores_closed_form_and_tie_break():
+    L, K, C = 40, 6, 5
+    w = wl.random_small(0, 1, L, K, C, ragged=False)
+    w.x[:] = 0
+    w.A[:] = 0
+    w.D[:] = 0
+    g = run_gpu(w)
+    N = [1] + [0] * L
+    for t in range(1, L + 1):
+        N[t] = C * sum(N[t - d] for d in range(1, min(K, t) + 1))
+    np.testing.assert_allclose(g["logZ"][0], math.log(N[L]), rtol=1e-13)
+    assert g["score"][0] == 0.0
+    assert np.all(g["labels"][0] == 0) and np.all(g["seg_start"][0] == 1)
+
+
+def test_genomic_full_size_invariants():
+    """Full genomic size: log Z against the oracle forward, plus invariants of the
+    gradients that hold at any size."""
+    w = wl.make_workload("genomic")
+    g = run_gpu(w)
+    assert g["status"] == 0
+    lz = oracle.logz(w.x, w.A, w.D, w.lengths)
+    assert abs(g["logZ"][0] - lz[0]) / abs(lz[0]) <= 1e-11
+    L = int(w.lengths[0])
+    dvec = np.arange(1, w.K + 1)[:, None]
+    np.testing.assert_allclose((dvec * g["dD"]).sum(), L, rtol=1e-10)         # total length
+    np.testing.assert_allclose(g["dD"].sum() - g["dA"].sum(), 1.0, atol=1e-6)  # segments - transitions
+    np.testing.assert_allclose(g["dX"][0, :L].sum(axis=1), 0.0, atol=1e-4)    # coverage sums to one
+    np.testing.assert_allclose(g["dX"][0].sum(axis=0), 0.0, atol=1e-2)        # zero mean per label
+    assert g["dA"].min() >= 0 and g["dD"].min() >= 0
