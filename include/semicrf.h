@@ -101,6 +101,23 @@ semicrf_status semicrf_prefix_scan(const semicrf_dims *dims, const float *x,
                                    void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * The same centring and prefix scan without a workspace, for callers that are
+ * given only their input and output buffers (a plugin or custom-op interface
+ * with no workspace hook) or that cannot call cudaMalloc under a fixed memory
+ * budget.  The pages have no counterpart to this entry point.
+ * Scratch: a library-owned static device array of 1 MiB (+256 bytes), held by
+ * every GPU that loads the library until exit; requires B*C <= 131072
+ * (SEMICRF_ERR_UNSUPPORTED_SHAPE otherwise).  Allocates nothing.  The first call
+ * on a device looks up the array's device address (make it before any stream
+ * capture).  All calls share the array: calls that overlap on the GPU race and
+ * must be serialised by the caller.  Device-side length errors are not
+ * reported by this entry point (such sequences are skipped).
+ */
+semicrf_status semicrf_prefix_scan_noalloc(const semicrf_dims *dims, const float *x,
+                                           const int32_t *lengths, double *S, double *nu,
+                                           void *stream);
+
+/*
  * Streaming forward (abstract: prefix-sum lookup instead of an edge tensor;
  * technical summary 2.B-2.C: O(K*C) ring of forward messages, normalised
  * checkpoints every ckpt_interval positions).  Writes logZ[b] and keeps the

@@ -18,7 +18,7 @@ from . import _lib
 from ._lib import (MAX_C, MAX_K, WS_SCAN, WS_TRAIN, WS_VITERBI, SemiCRFError, dims,
                    status_string)
 
-__all__ = ["workspace_bytes", "new_workspace", "prefix_scan", "forward", "backward", "viterbi",
+__all__ = ["workspace_bytes", "new_workspace", "prefix_scan", "prefix_scan_noalloc", "forward", "backward", "viterbi",
            "logz_and_grads", "device_status", "clear_device_status", "last_launch_count",
            "SemiCRFError", "status_string", "MAX_C", "MAX_K", "WS_TRAIN", "WS_VITERBI", "WS_SCAN",
            "load_library"]
@@ -82,6 +82,22 @@ def prefix_scan(x, lengths, ws=None, S=None, nu=None):
     d = dims(B, T, 1, C)
     _lib.check(_lib.load().semicrf_prefix_scan(ctypes.byref(d), _ptr(x), _ptr(lengths), _ptr(S), _ptr(nu),
                                                _ptr(ws), ws.numel(), _stream(x.device)), "prefix_scan")
+    return S, nu
+
+
+def prefix_scan_noalloc(x, lengths, S=None, nu=None):
+    """prefix_scan without a workspace: for callers that cannot allocate device
+    scratch.  Uses the library's fixed 1 MiB static scratch (B*C <= 131072);
+    concurrent calls on different streams race on it."""
+    torch = _torch()
+    B, T, C = x.shape
+    _need(x, torch.float32, (B, T, C), "x")
+    _need(lengths, torch.int32, (B,), "lengths")
+    S = torch.empty((B, T + 1, C), dtype=torch.float64, device=x.device) if S is None else S
+    nu = torch.empty((B, C), dtype=torch.float64, device=x.device) if nu is None else nu
+    d = dims(B, T, 1, C)
+    _lib.check(_lib.load().semicrf_prefix_scan_noalloc(ctypes.byref(d), _ptr(x), _ptr(lengths), _ptr(S),
+                                                       _ptr(nu), _stream(x.device)), "prefix_scan_noalloc")
     return S, nu
 
 

@@ -48,6 +48,7 @@ SIGNATURES = {
     "semicrf_workspace_bytes": (ctypes.c_size_t, [_DP, ctypes.c_int32]),
     "semicrf_check_dims": (ctypes.c_int, [_DP]),
     "semicrf_prefix_scan": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _S, _P]),
+    "semicrf_prefix_scan_noalloc": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P]),
     "semicrf_forward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _S, _P]),
     "semicrf_backward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P]),
     "semicrf_viterbi": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),

@@ -62,6 +62,8 @@ struct Layout {
 void prof_before(cudaStream_t st);
 void prof_after(cudaStream_t st);
 void prof_reset();
+// Sets what semicrf_last_launch_count reports for this thread.
+void record_launches(int n);
 
 Plan make_plan(int K, int C);
 bool make_layout(const semicrf_dims &d, int what, const Plan &p, Layout *out);
