@@ -112,7 +112,7 @@ def _speech(B, T, K, C, seed):
     t = np.arange(T)
     lo = np.maximum(t - 2, 0)
     hi = np.minimum(t + 3, T)
-    x = ((csum[:, hi, :] - csum[:, lo, :]) / (hi - lo)[None, :, None]).astype(np.float32)
+    x = np.ascontiguousarray(((csum[:, hi, :] - csum[:, lo, :]) / (hi - lo)[None, :, None]).astype(np.float32))
     A = _normal32(rng, (C, C), 0.3)
     d = np.arange(1, K + 1, dtype=np.float32)[:, None]
     D = (np.float32(-0.05) * d + _normal32(rng, (K, C), 0.1)).astype(np.float32)
