@@ -41,8 +41,9 @@ FP64_FMA_PER_SM_CLK = 64
 MUFU_PER_SM_CLK = 16
 HBM_FALLBACK_GBS = 6650.0
 SM_MAX_MHZ_FALLBACK = 1965.0
-KERNEL_NAMES = ["scan_partials", "scan_offsets", "scan_apply", "fwd_kernel", "fwd_recompute",
-                "bwd_kernel", "finalise_params", "finalise_dx"]
+# every kernel one step launches, in launch order (prefix_scan: 3, forward: 2, backward: 4)
+KERNEL_NAMES = ["scan_partials", "scan_offsets", "scan_apply", "exp_tables", "fwd_kernel",
+                "fwd_recompute", "bwd_kernel", "finalise_params", "finalise_dx"]
 
 
 def measured_peaks():
@@ -199,10 +200,10 @@ def run_gpu(args):
             lib.semicrf_set_profile_events(handles, 6)
         sc.prefix_scan(x, lens, ws=ws, S=S, nu=nu)
         if profile:
-            lib.semicrf_set_profile_events(ctypes_offset(handles, 6), 2)
+            lib.semicrf_set_profile_events(ctypes_offset(handles, 6), 4)
         sc.forward(S, A, D, lens, ws=ws, ckpt_interval=args.ckpt, logZ=logZ)
         if profile:
-            lib.semicrf_set_profile_events(ctypes_offset(handles, 8), 8)
+            lib.semicrf_set_profile_events(ctypes_offset(handles, 10), 8)
         sc.backward(S, A, D, lens, ws, ckpt_interval=args.ckpt, dX=dX, dA=dA, dD=dD)
         if profile:
             lib.semicrf_set_profile_events(None, 0)
@@ -344,7 +345,7 @@ def run_gpu(args):
                               "t_step_ms": ms, "frac_sfu": t_sfu * 1e3 / ms, "frac_fp64": t_fp64 * 1e3 / ms},
         "kernel_ms_per_step": {n: kern_ms[n] / args.steps for n in KERNEL_NAMES},
         "kernel_share": kern_share,
-        "gpu_launches": 8 * args.steps,
+        "gpu_launches": len(KERNEL_NAMES) * args.steps,
         "e2e": e2e,
         "clocks": clk,
         "wall_s": wall,

@@ -54,6 +54,27 @@ __device__ __forceinline__ void set_status(int32_t *status, int code)
     atomicCAS(reinterpret_cast<int *>(status), 0, code);
 }
 
+// 2^h with h clamped to the normal range [-1022, 1023] (branch free).
+__device__ __forceinline__ double pow2c(int h)
+{
+    h = max(-1022, min(1023, h));
+    return __longlong_as_double(static_cast<long long>(h + 1023) << 52);
+}
+
+// x * 2^h, exact unless the result over/underflows; |h| up to ~3000.
+__device__ __forceinline__ double scale2(double x, int h)
+{
+    while (h > 1000) {
+        x *= pow2(1000);
+        h -= 1000;
+    }
+    while (h < -1000) {
+        x *= pow2(-1000);
+        h += 1000;
+    }
+    return x * pow2(h);
+}
+
 // v mod K in [0, K) for any sign of v
 __device__ __forceinline__ int mod_pos(int v, int K)
 {

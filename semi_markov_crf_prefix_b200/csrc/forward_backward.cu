@@ -45,6 +45,8 @@
 // items in registers, and all-gathers the C values a'[t,:] through distributed
 // shared memory once per step.
 #include <math.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "device_util.cuh"
 #include "semicrf_internal.h"
@@ -184,6 +186,13 @@ __global__ void __launch_bounds__(kMaxThreads, 1) fwd_kernel(FbArgs a, KernelGeo
 
     double ap = 0.0;
     double St = ro.is_label ? Sb[(size_t)(t_begin + 1) * C + ro.c] : 0.0;
+    // recompute output is relative to Z: c0 = exp(-log sum a'_L), exponents minus k_L
+    int kZ = 0;
+    double c0 = 0.0;
+    if constexpr (RECOMPUTE) {
+        kZ = a.lz[b].k;
+        c0 = exp(-a.lz[b].logn);
+    }
     for (int t = t_begin + 1; t <= t_end; ++t) {
         const int par = t & 1;
         // next step's S row, fetched a step ahead
@@ -234,8 +243,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1) fwd_kernel(FbArgs a, KernelGeo
             }
             if (RECOMPUTE) {
                 size_t row = ((size_t)b * (a.T + 1) + t) * C;
-                if (ro.is_label) a.aA[row + ro.c] = ap;
-                if (rank == 0 && ro.tid == 0) a.aK[(size_t)b * (a.T + 1) + t] = k;
+                if (ro.is_label) a.cA[row + ro.c] = ap * c0;
+                if (rank == 0 && ro.tid == 0) a.eA[(size_t)b * (a.T + 1) + t] = k - kZ;
             }
             break;
         }
@@ -269,12 +278,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1) fwd_kernel(FbArgs a, KernelGeo
             ring[(t % K) * Cg + ro.lc] = U;
             if constexpr (RECOMPUTE) {
                 size_t row = ((size_t)b * (a.T + 1) + t) * C + ro.c;
-                a.aU[row] = U;
-                a.aA[row] = ap;
-                a.aR[row] = r;
+                a.cU[row] = U * c0;
+                a.cA[row] = ap * c0;
+                a.eU[row] = r - kZ;
             }
         }
-        if (RECOMPUTE && rank == 0 && ro.tid == 0) a.aK[(size_t)b * (a.T + 1) + t] = k;
+        if (RECOMPUTE && rank == 0 && ro.tid == 0) a.eA[(size_t)b * (a.T + 1) + t] = k - kZ;
         if (!RECOMPUTE && (t % a.delta) == 0) {
             // checkpoint t / delta: ring after step t, r, k_{t+1}
             __syncthreads();
@@ -330,7 +339,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) bwd_kernel(FbArgs a, KernelGeo
     const double *Sb = a.S + (size_t)b * (a.T + 1) * C;
     const size_t rowbase = (size_t)b * (a.T + 1);
     const int kZ = a.lz[b].k;
-    const double lognZ = a.lz[b].logn;
+    const double c0 = exp(-a.lz[b].logn);   // 1/sum_c a'[L,c]
 
     double W[DPT], E[CPT], accA[CPT];
 #pragma unroll
@@ -364,16 +373,14 @@ __global__ void __launch_bounds__(kMaxThreads, 1) bwd_kernel(FbArgs a, KernelGeo
         rb = (int)rint(SL / kLn2);
         ring[(L % K) * Cg + ro.lc] = exp(SL - kLn2 * (double)rb);
         // coverage of position L-1: P(the last segment has label c) = a'[L,c] / sum a'[L,:]
-        const double apL = a.aA[(rowbase + L) * C + ro.c];
-        const int kL = a.aK[rowbase + L];
-        mu_acc = apL * exp(kLn2 * (double)(kL - kZ) - lognZ);
+        mu_acc = scale2(a.cA[(rowbase + L) * C + ro.c], a.eA[rowbase + L]);
         const int s = L - 1;
         if (s == 0) {
-            coef[ro.lc] = exp(kLn2 * (double)(rb - kZ) - lognZ);
+            coef[ro.lc] = scale2(c0, rb - kZ);
         } else {
             const size_t row = (rowbase + s) * C + ro.c;
-            coef[ro.lc] = a.aU[row] * exp(kLn2 * (double)(a.aR[row] + rb - kZ) - lognZ);
-            a2[ro.lc] = a.aA[row] * exp(kLn2 * (double)(a.aK[rowbase + s] + kb - kZ) - lognZ);
+            coef[ro.lc] = scale2(a.cU[row], a.eU[row] + rb);
+            a2[ro.lc] = scale2(a.cA[row], a.eA[rowbase + s] + kb);
         }
     }
     if constexpr (CLUSTER) cluster_barrier();
@@ -390,10 +397,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1) bwd_kernel(FbArgs a, KernelGeo
             St_next = Sb[(size_t)(s - 1) * C + ro.c];
             if (s - 1 >= 1) {
                 const size_t row = (rowbase + s - 1) * C + ro.c;
-                nU = a.aU[row];
-                nA = a.aA[row];
-                nR = a.aR[row];
-                nK = a.aK[rowbase + s - 1];
+                nU = a.cU[row];
+                nA = a.cA[row];
+                nR = a.eU[row];
+                nK = a.eA[rowbase + s - 1];
             }
         }
         // (A) pb share and dD accumulation over this thread's durations
@@ -482,11 +489,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1) bwd_kernel(FbArgs a, KernelGeo
             musum += mu_acc;
             mu_acc += end - start;
             if (s - 1 == 0) {
-                coef[ro.lc] = exp(kLn2 * (double)(rb - kZ) - lognZ);
+                coef[ro.lc] = scale2(c0, rb - kZ);
                 a2[ro.lc] = 0.0;
             } else {
-                coef[ro.lc] = nU * exp(kLn2 * (double)(nR + rb - kZ) - lognZ);
-                a2[ro.lc] = nA * exp(kLn2 * (double)(nK + kbn - kZ) - lognZ);
+                coef[ro.lc] = scale2(nU, nR + rb);
+                a2[ro.lc] = scale2(nA, nK + kbn);
             }
         }
         kb = kbn;
@@ -636,23 +643,48 @@ FbLauncher pick(const Plan &p)
 
 }  // namespace
 
+// Which kernel family runs: the warp-per-sequence kernels when the shape allows,
+// else the cluster kernels.  SEMICRF_KERNEL_PATH=general forces the cluster
+// kernels (used by the tests to keep both families under parity checks).
+bool use_small(int K, int C)
+{
+    const char *env = getenv("SEMICRF_KERNEL_PATH");
+    if (env && strcmp(env, "general") == 0) return false;
+    return small_path_ok(K, C);
+}
+
 cudaError_t launch_forward(const Plan &p, const FbArgs &a, cudaStream_t st, int *launches)
 {
-    FbLauncher f = pick(p);
-    if (!f) return cudaErrorInvalidConfiguration;
-    cudaError_t e = f(p, a, st, 0);
+    cudaError_t e = launch_exp_tables(a, st);
+    if (e != cudaSuccess) return e;
+    *launches += 1;
+    if (use_small(a.K, a.C)) {
+        e = launch_small(a, st, 0);
+    } else {
+        FbLauncher f = pick(p);
+        if (!f) return cudaErrorInvalidConfiguration;
+        e = f(p, a, st, 0);
+    }
     if (e == cudaSuccess) *launches += 1;
     return e;
 }
 
 cudaError_t launch_backward(const Plan &p, const FbArgs &a, cudaStream_t st, int *launches)
 {
-    FbLauncher f = pick(p);
-    if (!f) return cudaErrorInvalidConfiguration;
-    cudaError_t e = f(p, a, st, 1);   // recompute every checkpoint segment
-    if (e != cudaSuccess) return e;
-    e = f(p, a, st, 2);               // backward with marginals
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
+    if (use_small(a.K, a.C)) {
+        e = launch_small(a, st, 1);   // recompute every checkpoint segment
+        if (e != cudaSuccess) return e;
+        e = launch_small(a, st, 2);   // backward with marginals
+        if (e != cudaSuccess) return e;
+    } else {
+        FbLauncher f = pick(p);
+        if (!f) return cudaErrorInvalidConfiguration;
+        e = f(p, a, st, 1);   // recompute every checkpoint segment
+        if (e != cudaSuccess) return e;
+        e = f(p, a, st, 2);   // backward with marginals
+        if (e != cudaSuccess) return e;
+    }
     const int nparam = a.C * a.C + a.K * a.C;
     prof_before(st);
     finalise_params<<<(nparam + 255) / 256, 256, 0, st>>>(a);

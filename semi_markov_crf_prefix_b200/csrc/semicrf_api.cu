@@ -109,10 +109,13 @@ bool make_layout(const semicrf_dims &d, int what, const Plan &p, Layout *out)
         L.logz = take(B * sizeof(LogZState));
         L.ckpt_stride = align_up(K * C * 8 + (C + 1) * 4, 256);
         L.ckpt = take(B * (size_t)L.J * L.ckpt_stride);
-        L.aU = take(B * (T + 1) * C * 8);
-        L.aA = take(B * (T + 1) * C * 8);
-        L.aR = take(B * (T + 1) * C * 4);
-        L.aK = take(B * (T + 1) * 4);
+        L.tES = take(B * (T + 1) * C * 8);
+        L.tIES = take(B * (T + 1) * C * 8);
+        L.tM = take(B * (T + 1) * C * 4);
+        L.cU = take(B * (T + 1) * C * 8);
+        L.cA = take(B * (T + 1) * C * 8);
+        L.eU = take(B * (T + 1) * C * 4);
+        L.eA = take(B * (T + 1) * 4);
         L.accD = take(B * K * C * 8);
         L.accA = take(B * C * C * 8);
         L.musum = take(B * C * 8);
@@ -187,10 +190,13 @@ FbArgs fb_args(const semicrf_dims *d, const Layout &lay, void *ws)
     a.lz = at<LogZState>(ws, lay.logz);
     a.ckpt = at<unsigned char>(ws, lay.ckpt);
     a.ckpt_stride = lay.ckpt_stride;
-    a.aU = at<double>(ws, lay.aU);
-    a.aA = at<double>(ws, lay.aA);
-    a.aR = at<int32_t>(ws, lay.aR);
-    a.aK = at<int32_t>(ws, lay.aK);
+    a.tES = at<double>(ws, lay.tES);
+    a.tIES = at<double>(ws, lay.tIES);
+    a.tM = at<int32_t>(ws, lay.tM);
+    a.cU = at<double>(ws, lay.cU);
+    a.cA = at<double>(ws, lay.cA);
+    a.eU = at<int32_t>(ws, lay.eU);
+    a.eA = at<int32_t>(ws, lay.eA);
     a.accD = at<double>(ws, lay.accD);
     a.accA = at<double>(ws, lay.accA);
     a.musum = at<double>(ws, lay.musum);

@@ -43,10 +43,17 @@ struct Layout {
     size_t logz = 0;        // LogZState [B]
     size_t ckpt = 0;        // [B][J] records of ckpt_stride bytes
     size_t ckpt_stride = 0; // ring double[K*C], r int32[C], k int32
-    size_t aU = 0;          // double [B][T+1][C]   recomputed ring rows
-    size_t aA = 0;          // double [B][T+1][C]   recomputed scaled alpha
-    size_t aR = 0;          // int32  [B][T+1][C]   ring exponent per row
-    size_t aK = 0;          // int32  [B][T+1]      alpha exponent per position
+    // Recomputed forward quantities per position t and label c, as mantissa and
+    // power-of-two exponent relative to Z:
+    //   exp(at[t,c] - S[t,c] - log Z) = cU * 2^eU,   exp(al[t,c] - log Z) = cA * 2^eA
+    // exp(S[t,c]) split as es * 2^m with |log es| <= ln2/2 (es, 1/es, m per position)
+    size_t tES = 0;         // double [B][T+1][C]  exp(s)
+    size_t tIES = 0;        // double [B][T+1][C]  exp(-s)
+    size_t tM = 0;          // int32  [B][T+1][C]  m
+    size_t cU = 0;          // double [B][T+1][C]
+    size_t cA = 0;          // double [B][T+1][C]
+    size_t eU = 0;          // int32  [B][T+1][C]
+    size_t eA = 0;          // int32  [B][T+1]
     size_t accD = 0;        // double [B][K][C]
     size_t accA = 0;        // double [B][C][C]
     size_t musum = 0;       // double [B][C]
@@ -89,13 +96,22 @@ struct FbArgs {
     LogZState *lz;
     unsigned char *ckpt;
     size_t ckpt_stride;
-    double *aU, *aA;
-    int32_t *aR, *aK;
+    double *cU, *cA;
+    int32_t *eU, *eA;
+    double *tES, *tIES;
+    int32_t *tM;
     double *accD, *accA, *musum, *mures, *logzb;
     float *dX;
     double *dA, *dD;
     int32_t *status;
 };
+// Warp-per-sequence kernels for C <= 32, K <= 32 (kind 0 forward, 1 recompute, 2 backward).
+bool small_path_ok(int K, int C);
+cudaError_t launch_small(const FbArgs &a, cudaStream_t st, int kind);
+
+// exp tables of S (tES, tIES, tM) for every position; fully parallel, HBM-bound.
+cudaError_t launch_exp_tables(const FbArgs &a, cudaStream_t st);
+
 cudaError_t launch_forward(const Plan &p, const FbArgs &a, cudaStream_t st, int *launches);
 cudaError_t launch_backward(const Plan &p, const FbArgs &a, cudaStream_t st, int *launches);
 

@@ -102,6 +102,28 @@ def test_named_small(name):
     check_against_oracle(w, run_gpu(w))
 
 
+@pytest.mark.parametrize("name", ["tiny", "ner"])
+def test_named_small_cluster_kernels(name, monkeypatch):
+    # the same workloads through the cluster kernels instead of the warp-per-sequence ones
+    monkeypatch.setenv("SEMICRF_KERNEL_PATH", "general")
+    w = wl.make_workload(name)
+    check_against_oracle(w, run_gpu(w))
+
+
+def test_kernel_families_agree():
+    import os
+    w = wl.make_workload("ner", B=8)
+    a = run_gpu(w)
+    os.environ["SEMICRF_KERNEL_PATH"] = "general"
+    try:
+        b = run_gpu(w)
+    finally:
+        del os.environ["SEMICRF_KERNEL_PATH"]
+    np.testing.assert_allclose(a["logZ"], b["logZ"], rtol=1e-13)
+    for k in ("dX", "dA", "dD"):
+        np.testing.assert_allclose(a[k], b[k], atol=1e-9, rtol=1e-12)
+
+
 def test_upstream_weights():
     w = wl.make_workload("ner")
     grad = np.random.default_rng(1).normal(size=w.B)
@@ -124,7 +146,9 @@ def test_large_reduced_T():
     check_against_oracle(w, run_gpu(w))
 
 
-@pytest.mark.parametrize("seed,B,T,K,C", [(0, 3, 37, 5, 3), (1, 5, 100, 1, 7), (2, 2, 70, 70, 2),
+@pytest.mark.parametrize("seed,B,T,K,C", [(8, 9, 90, 32, 32), (9, 6, 130, 24, 9), (10, 5, 64, 31, 1),
+                                           (11, 7, 200, 2, 31), (12, 3, 40, 17, 24),
+                                           (0, 3, 37, 5, 3), (1, 5, 100, 1, 7), (2, 2, 70, 70, 2),
                                            (3, 4, 129, 33, 33), (4, 1, 1, 4, 5), (5, 2, 50, 200, 9),
                                            (6, 3, 300, 40, 64), (7, 2, 200, 300, 20)])
 def test_random_shapes(seed, B, T, K, C):
