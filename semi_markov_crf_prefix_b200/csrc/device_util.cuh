@@ -75,6 +75,34 @@ __device__ __forceinline__ double scale2(double x, int h)
     return x * pow2(h);
 }
 
+// x * 2^h for |h| <= 2044 without branches (two exact power-of-two factors).
+__device__ __forceinline__ double scale2c(double x, int h)
+{
+    const int h1 = h / 2;
+    return (x * pow2c(h1)) * pow2c(h - h1);
+}
+
+// Asynchronous global -> shared copies (Ampere-and-later cp.async), grouped.
+__device__ __forceinline__ void cp_async8(void *smem, const void *gmem)
+{
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(s), "l"(gmem) : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(void *smem, const void *gmem)
+{
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(s), "l"(gmem) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // v mod K in [0, K) for any sign of v
 __device__ __forceinline__ int mod_pos(int v, int K)
 {

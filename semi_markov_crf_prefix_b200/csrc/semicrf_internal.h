@@ -11,8 +11,11 @@
 namespace semicrf {
 
 // Ring columns are rebased (scaled by an exact power of two) when the weighted
-// column sum leaves [2^-kRebaseBits, 2^kRebaseBits].
-constexpr int kRebaseBits = 256;
+// column sum leaves [2^-kRebaseBits, 2^kRebaseBits].  Within one step a column's
+// newest entry moves by a bounded factor (transition, duration and one emission
+// term), so with 512 bits every product formed in a step stays far inside the
+// float64 range (2^+-1022).
+constexpr int kRebaseBits = 512;
 constexpr int kMaxThreads = 512;
 constexpr size_t kSmemBudget = 220 * 1024;
 

@@ -120,8 +120,10 @@ def test_kernel_families_agree():
     finally:
         del os.environ["SEMICRF_KERNEL_PATH"]
     np.testing.assert_allclose(a["logZ"], b["logZ"], rtol=1e-13)
-    for k in ("dX", "dA", "dD"):
+    for k in ("dA", "dD"):
         np.testing.assert_allclose(a[k], b[k], atol=1e-9, rtol=1e-12)
+    # dX is float32: a float64 difference of ~1e-15 may flip one float32 rounding
+    np.testing.assert_allclose(a["dX"], b["dX"], atol=2e-7, rtol=0)
 
 
 def test_upstream_weights():
