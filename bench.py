@@ -55,6 +55,27 @@ def measured_peaks():
         return None
 
 
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from the last ncu capture of this kernel (profiles/
+    dram_traffic.txt), or None when the kernel source changed since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    for line in lines:
+        f = line.split()
+        if len(f) != 5 or line.startswith("#") or f[0] != kernel or f[1] != workload:
+            continue
+        try:
+            src = open(os.path.join(ROOT, f[3]), "rb").read()
+        except OSError:
+            return None
+        return int(f[2]) if hashlib.sha256(src).hexdigest()[:16] == f[4] else None
+    return None
+
+
 def algorithmic(w):
     """Terms and bytes the method must do (not the recompute it chooses to do)."""
     sumL = int(w.lengths.astype(np.int64).sum())
@@ -315,7 +336,8 @@ def run_gpu(args):
     if dom in work_flop:
         achieved = work_flop[dom] / (per_launch_ms / 1e3) / 1e12
         roof = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": fp64_peak_tflops,
-                "unit": "TFLOP/s", "frac": achieved / fp64_peak_tflops, "traffic": None,
+                "unit": "TFLOP/s", "frac": achieved / fp64_peak_tflops,
+                "traffic": recorded_traffic(dom, args.config),
                 "peak_source": f"derived: {N_SM} SMs x {FP64_FMA_PER_SM_CLK} FP64 FMA/clk x 2 x {sm_max:.0f} MHz",
                 "work": "2 flop per (log-sum-exp, +) term: sum_b L_b (K*C + C*C) terms per launch"}
     else:
