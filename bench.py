@@ -179,6 +179,7 @@ def run_gpu(args):
     import torch.distributed as dist
     import semi_markov_crf_prefix_b200 as sc
     from semi_markov_crf_prefix_b200 import _lib
+    from semi_markov_crf_prefix_b200.dist import reduce_param_grads
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -190,7 +191,10 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     sc.load_library()
 
-    w = wl.make_workload(args.config, seed=args.seed + rank)
+    w = wl.make_workload(args.config, seed=args.seed)
+    if rank > 0:   # data-parallel: every rank its own emissions and lengths, shared A and D
+        own = wl.make_workload(args.config, seed=args.seed + 1000 * rank)
+        w.x, w.lengths = own.x, own.lengths
     B, T, K, C = w.B, w.T, w.K, w.C
     sumL, terms_pass, bytes_path = algorithmic(w)
     stream = torch.cuda.current_stream(dev)
@@ -229,8 +233,7 @@ def run_gpu(args):
         if profile:
             lib.semicrf_set_profile_events(None, 0)
         if world > 1:
-            dist.all_reduce(dA)
-            dist.all_reduce(dD)
+            reduce_param_grads(dA, dD)
 
     sc.clear_device_status(ws)
     for _ in range(args.warmup):
