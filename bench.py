@@ -41,9 +41,13 @@ FP64_FMA_PER_SM_CLK = 64
 MUFU_PER_SM_CLK = 16
 HBM_FALLBACK_GBS = 6650.0
 SM_MAX_MHZ_FALLBACK = 1965.0
-# every kernel one step launches, in launch order (prefix_scan: 3, forward: 2, backward: 4)
-KERNEL_NAMES = ["scan_partials", "scan_offsets", "scan_apply", "exp_tables", "fwd_kernel",
-                "fwd_recompute", "bwd_kernel", "finalise_params", "finalise_dx"]
+# every kernel one step launches, in launch order: prefix_scan 3, forward 2, and a
+# backward of 4 (warp-per-sequence kernels, C, K <= 32) or 6 (cluster kernels, whose
+# dD and dA are separate contraction kernels)
+SCAN_NAMES = ["scan_partials", "scan_offsets", "scan_apply"]
+FWD_NAMES = ["exp_tables", "fwd_kernel"]
+BWD_NAMES = {4: ["fwd_recompute", "bwd_kernel", "finalise_params", "finalise_dx"],
+             6: ["fwd_recompute", "bwd_kernel", "dur_grad", "trans_grad", "finalise_params", "finalise_dx"]}
 
 
 def measured_peaks():
@@ -212,6 +216,13 @@ def run_gpu(args):
     dD = torch.empty((K, C), dtype=torch.float64, device=dev)
     flush = torch.empty(256 * 2**20 // 4, dtype=torch.float32, device=dev)
 
+    # the backward's kernel list depends on the kernel family the shape uses
+    sc.clear_device_status(ws)
+    sc.prefix_scan(x, lens, ws=ws, S=S, nu=nu)
+    sc.forward(S, A, D, lens, ws=ws, ckpt_interval=args.ckpt, logZ=logZ)
+    sc.backward(S, A, D, lens, ws, ckpt_interval=args.ckpt, dX=dX, dA=dA, dD=dD)
+    n_bwd = sc.last_launch_count()
+    KERNEL_NAMES = SCAN_NAMES + FWD_NAMES + BWD_NAMES[n_bwd]
     # per-kernel events (recorded by the library around each launch)
     n_ev = 2 * len(KERNEL_NAMES)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
@@ -228,7 +239,7 @@ def run_gpu(args):
             lib.semicrf_set_profile_events(ctypes_offset(handles, 6), 4)
         sc.forward(S, A, D, lens, ws=ws, ckpt_interval=args.ckpt, logZ=logZ)
         if profile:
-            lib.semicrf_set_profile_events(ctypes_offset(handles, 10), 8)
+            lib.semicrf_set_profile_events(ctypes_offset(handles, 10), 2 * n_bwd)
         sc.backward(S, A, D, lens, ws, ckpt_interval=args.ckpt, dX=dX, dA=dA, dD=dD)
         if profile:
             lib.semicrf_set_profile_events(None, 0)

@@ -1,0 +1,1074 @@
+// fb_cluster.cu -- latency-first forward, recompute and backward chains for any K
+// and C within the compiled limits: one thread-block cluster per sequence (per
+// checkpoint segment when recomputing), labels split across its G CTAs.
+//
+// Same recursions and scaled exp-space representation as forward_backward.cu
+// (Streaming Structured Inference with Flash-SemiCRF, abstract; technical
+// summary 2.A-2.C).  A CTA has three kinds of warps.  Owner warps run the chain
+// of one label per lane; transition warps form the C x C product; window warps
+// form the duration sums.  The sequential chain of one position is
+//   owners:      p = U[t-1] W0 + pre_t ;  a'[t,c] = p e ; st.async of a'[t,c]
+//                into every CTA of the cluster, completing bytes on that CTA's
+//                mbarrier for the position (G = 1: a plain store + bar.arrive)
+//   transition:  wait for the C values, q[c] = sum_c' a'[t,c'] exp(A[c',c])
+//                (LPL lanes per label, CPL terms each, shuffle reduction; the
+//                same pass sums n_t = sum_c' a'[t,c'] for the normaliser);
+//                bar.arrive to the owners
+//   owners:      bar.sync, U[t,c] = q f, the new ring row
+//   all:         one bar.sync (with an OR of the timeout flags) per position
+// Work off the chain:
+//  * window warps form the duration sum over d >= 3 two positions ahead,
+//      pre3_{t+2} = sum_{d=3..K} U[t+2-d] exp(D[d-1]),
+//    starting right after the previous position's barrier, in parallel with
+//    the owners and the exchange.  They read the rows at the reference of
+//    position t-1 and bring them there themselves (a rebase of a column at t-1
+//    rescales every stored row of it by the same power of two, exactly); the
+//    owner scales pre3 by the rebases of the two positions in between.
+//  * the ring holds every row twice (slots r mod K and r mod K + K), so the
+//    K - 2 rows of a window are contiguous and need no wrap arithmetic.
+//  * the normaliser is pipelined: k_{t+2} = k_t + floor(log2 n_t) is formed in
+//    every CTA from the same sum in the same order and used two positions
+//    later; log Z = ln2 k_L + log n_L stays exact.
+//  * exp(S) comes from the exp tables, prefetched with cp.async by the owners.
+// The backward chain computes beta only and stores, per position, the rows the
+// parameter gradients need (V, its reference, the normalised beta and the
+// backward normaliser); dA and dD are then dense contractions over all
+// positions done by cl_grads.cu on the whole GPU.  The coverage marginal and
+// dX stay on the chain (one running sum per label).
+// Every wait is bounded: a wait that runs out sets SEMICRF_ERR_DEVICE_TIMEOUT,
+// the end-of-position barrier ORs the flag over the CTA and the whole CTA leaves
+// its loop; the other CTAs of the cluster then run out too and all meet at the
+// final cluster barrier.  Buffers of a position are indexed by the step count u
+// (0 for the first position the kernel runs), so mbarrier phases start at 0.
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
+
+#include "device_util.cuh"
+#include "semicrf_internal.h"
+
+namespace semicrf {
+namespace {
+
+constexpr int kPF = 8;                        // exp-table prefetch ring depth (positions)
+constexpr long long kWaitCycles = 1ll << 31;  // ~1 s at 2 GHz
+
+__device__ __forceinline__ void cta_barrier(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ void cta_arrive(int id, int nthreads)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// bar.sync with an OR over the threads' flags: every thread gets the same answer
+__device__ __forceinline__ bool cta_barrier_or(int id, int nthreads, bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, int count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, int bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait (bounded) for the completion of the mbarrier phase of the given parity.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+{
+    const uint32_t a = smem_addr(bar);
+    if (mbar_try(a, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try(a, parity))
+        if (clock64() - t0 > kWaitCycles) return false;
+    return true;
+}
+
+// Store v at the address of `local` in CTA `rank` of the cluster and complete 8
+// bytes on that CTA's copy of `bar`.
+__device__ __forceinline__ void st_async_f64(const double *local, const uint64_t *bar, uint32_t rank, double v)
+{
+    uint32_t ra, rb;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_addr(local)), "r"(rank));
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(smem_addr(bar)), "r"(rank));
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];" ::"r"(ra),
+                 "l"(__double_as_longlong(v)), "r"(rb)
+                 : "memory");
+}
+
+// xor-shuffle sum over groups of `width` consecutive lanes (width a power of two <= 32)
+__device__ __forceinline__ double group_sum(double v, int width)
+{
+    for (int off = width >> 1; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+// x * 2^h, with the common h = 0 free
+__device__ __forceinline__ double rescale(double x, int h) { return h == 0 ? x : scale2c(x, h); }
+
+// Shared memory of both chains (the backward uses the pf_cu/pf_ca/pf_eu/pf_ea rings).
+struct ClSmem {
+    double *ring;    // [2K][RS] every row twice
+    double *Wd;      // [K][RS]  exp(D)
+    double *gath;    // [2][C]   a' (forward) or bp (backward) of the position, all labels
+    double *qbuf;    // [Cg]     transition result of each label, for its owner
+    double *pre3;    // [4][Cg][PW] window sums two positions ahead
+    double *pf_es, *pf_ies, *pf_cu, *pf_ca;   // [kPF][Cg] prefetch rings
+    uint64_t *full;  // [2] exchange mbarriers
+    int *pf_m, *pf_eu, *pf_ea;                // [kPF][Cg] each
+    int *hbuf;       // [2][Cg] rebase exponent of each label at the last two positions
+    int *kbuf;       // [4]     normaliser exponents
+};
+
+__host__ __device__ __forceinline__ size_t cl_smem_bytes_impl(int K, int C, const ClGeom &g, bool bwd)
+{
+    const size_t npf = bwd ? 4 : 2;
+    const size_t nd = 3 * (size_t)K * g.RS + 2 * (size_t)C + g.Cg + 4 * (size_t)g.Cg * g.PW + npf * kPF * g.Cg;
+    const size_t ni = (bwd ? 3 : 1) * (size_t)kPF * g.Cg + 2 * (size_t)g.Cg + 4;
+    return nd * sizeof(double) + 2 * sizeof(uint64_t) + ni * sizeof(int);
+}
+
+__device__ __forceinline__ ClSmem cl_smem(double *base, int K, int C, const ClGeom &g, bool bwd)
+{
+    ClSmem s;
+    s.ring = base;
+    s.Wd = s.ring + 2 * (size_t)K * g.RS;
+    s.gath = s.Wd + (size_t)K * g.RS;
+    s.qbuf = s.gath + 2 * C;
+    s.pre3 = s.qbuf + g.Cg;
+    s.pf_es = s.pre3 + 4 * g.Cg * g.PW;
+    s.pf_ies = s.pf_es + kPF * g.Cg;
+    s.pf_cu = s.pf_ies + kPF * g.Cg;
+    s.pf_ca = bwd ? s.pf_cu + kPF * g.Cg : s.pf_cu;
+    double *dend = bwd ? s.pf_ca + kPF * g.Cg : s.pf_cu;
+    s.full = reinterpret_cast<uint64_t *>(dend);
+    s.pf_m = reinterpret_cast<int *>(s.full + 2);
+    s.pf_eu = s.pf_m + kPF * g.Cg;
+    s.pf_ea = bwd ? s.pf_eu + kPF * g.Cg : s.pf_eu;
+    s.hbuf = bwd ? s.pf_ea + kPF * g.Cg : s.pf_eu;
+    s.kbuf = s.hbuf + 2 * g.Cg;
+    return s;
+}
+
+// sum_i a[i] b[i] as a pairwise tree (products in parallel, log2 N levels of adds):
+// with FP64 latency in the tens of cycles, depth matters more than op count.
+template <int N>
+__device__ __forceinline__ double tree_dot(const double (&x)[N], const double (&y)[N])
+{
+    static_assert(N >= 2 && (N & (N - 1)) == 0, "N must be a power of two");
+    double p[N / 2];
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) p[i] = fma(x[2 * i], y[2 * i], x[2 * i + 1] * y[2 * i + 1]);
+#pragma unroll
+    for (int w = N / 2; w > 1; w >>= 1) {
+#pragma unroll
+        for (int i = 0; i < w / 2; ++i) p[i] = p[2 * i] + p[2 * i + 1];
+    }
+    return p[0];
+}
+
+// Sum of n rows spaced `step` doubles apart from u (downwards when dir < 0)
+// times weights spaced `step` apart from w (upwards), eight rows per chunk: all
+// sixteen loads of a chunk issue together, then a product tree.
+__device__ __forceinline__ double strided_dot(const double *u, int ustep, const double *w, int wstep, int n)
+{
+    double acc = 0.0;
+#pragma unroll 2
+    for (int m0 = 0; m0 < n; m0 += 8) {
+        double v[8], x[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const bool ok = m0 + i < n;
+            v[i] = ok ? u[(m0 + i) * ustep] : 0.0;
+            x[i] = ok ? w[(m0 + i) * wstep] : 0.0;
+        }
+        acc += tree_dot<8>(v, x);
+    }
+    return acc;
+}
+
+// Forward window: sum over d = d0 + m*LPW <= K (d0 = 3 + j) of ring row (tau - d)
+// times exp(D[d-1]) for label lc, with tau mod K = tauK.  Rows with d >= 4 are
+// first brought to the reference of position tau - 3 (multiplied by 2^hp, both
+// copies); row tau - 3 (d = 3) was written at that reference.
+__device__ __forceinline__ double window_fwd(double *ring, const double *Wd, int K, int RS, int lc, int LPW, int j,
+                                             int tauK, int hp)
+{
+    const int d0 = 3 + j;
+    if (d0 > K) return 0.0;
+    const int n = (K - d0) / LPW + 1;
+    const int step = LPW * RS;
+    if (hp != 0) {
+        for (int m = 0; m < n; ++m) {
+            const int d = d0 + m * LPW;
+            if (d < 4) continue;
+            const int sl = tauK + K - d;
+            const int other = sl >= K ? sl - K : sl + K;
+            const double v = rescale(ring[sl * RS + lc], hp);
+            ring[sl * RS + lc] = v;
+            ring[other * RS + lc] = v;
+        }
+    }
+    // the copy whose slots fall in [0, 2K): rows tau - d at slot tauK + K - d
+    return strided_dot(ring + (size_t)(tauK + K - d0) * RS + lc, -step, Wd + (size_t)(d0 - 1) * RS + lc, step, n);
+}
+
+// Backward window: sum over i = i0 + m*LPW <= K-2 (i0 = 1 + j) of ring row (s + i)
+// times exp(D[i+1]) (position s-2, duration i+2), s mod K = sK.  Rows with i >= 2
+// are first brought to the reference of position s+1 (multiplied by 2^hp).
+__device__ __forceinline__ double window_bwd(double *ring, const double *Wd, int K, int RS, int lc, int LPW, int j,
+                                             int sK, int hp)
+{
+    const int i0 = 1 + j;
+    if (i0 > K - 2) return 0.0;
+    const int n = (K - 2 - i0) / LPW + 1;
+    const int step = LPW * RS;
+    if (hp != 0) {
+        for (int m = 0; m < n; ++m) {
+            const int i = i0 + m * LPW;
+            if (i < 2) continue;
+            const int sl = sK + i;
+            const int other = sl >= K ? sl - K : sl + K;
+            const double v = rescale(ring[sl * RS + lc], hp);
+            ring[sl * RS + lc] = v;
+            ring[other * RS + lc] = v;
+        }
+    }
+    return strided_dot(ring + (size_t)(sK + i0) * RS + lc, step, Wd + (size_t)(i0 + 1) * RS + lc, step, n);
+}
+
+// Normaliser sum n = sum_c g[c] over one warp: C/32 loads per lane, a tree, five
+// shuffle levels.  Every lane gets n; every CTA forms it in the same order.
+__device__ __forceinline__ double warp_total(const double *g, int C, int lane)
+{
+    double acc = 0.0;
+    for (int i0 = 0; i0 < C; i0 += 128) {
+        double v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int i = i0 + 32 * k + lane;
+            v[k] = i < C ? g[i] : 0.0;
+        }
+        acc += (v[0] + v[1]) + (v[2] + v[3]);
+    }
+    return group_sum(acc, 32);
+}
+
+// Roles of a thread: owner warps (label lc = lane of the warp's 32), then
+// transition warps (LPL lanes per label), then window warps (LPW lanes per label).
+struct Roles {
+    bool is_own, is_tr, is_win, lab_ok;
+    int lc, j, c;
+};
+
+__device__ __forceinline__ Roles cl_roles(const ClGeom &g, int warp, int lane, int c0l, int cg_own)
+{
+    Roles r;
+    r.is_own = warp < g.NWO;
+    r.is_tr = !r.is_own && warp < g.NWO + g.NWT;
+    r.is_win = !r.is_own && !r.is_tr && warp < g.NWO + g.NWT + g.NWW;
+    r.lc = 0;
+    r.j = 0;
+    if (r.is_own) {
+        r.lc = warp * 32 + lane;
+    } else if (r.is_tr) {
+        const int tl = (warp - g.NWO) * 32 + lane;
+        r.lc = tl / g.LPL;
+        r.j = tl % g.LPL;
+    } else if (r.is_win) {
+        const int wl = (warp - g.NWO - g.NWT) * 32 + lane;
+        r.lc = wl / g.LPW;
+        r.j = wl % g.LPW;
+    }
+    r.lab_ok = (r.is_own || r.is_tr || r.is_win) && r.lc < cg_own;
+    r.c = c0l + (r.lab_ok ? r.lc : 0);
+    return r;
+}
+
+// Waits of the transition warps and of owner warp 0 (which forms the normaliser)
+// for the C values of a position: the mbarrier of the cluster exchange, or with
+// one CTA a named barrier after the owners' plain stores.
+template <bool CLUSTER>
+__device__ __forceinline__ bool wait_values(ClSmem &sm, int par, int u, bool skip)
+{
+    if constexpr (CLUSTER) {
+        if (skip) return true;
+        return mbar_wait(&sm.full[par], (u >> 1) & 1);
+    } else {
+        return true;
+    }
+}
+
+template <int CPL, int MAXT, bool CLUSTER, bool RECOMPUTE>
+__global__ void __launch_bounds__(MAXT, 1) cl_fwd_kernel(FbArgs a, ClGeom g)
+{
+    extern __shared__ __align__(16) double smc[];
+    const int K = a.K, C = a.C, Cg = g.Cg, NT = g.NT, RS = g.RS, PW = g.PW;
+    const int NOT = 32 * (g.NWO + g.NWT);   // owner + transition threads
+    const int W0T = 32 * (g.NWO + g.NWT);   // first window thread
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rank = CLUSTER ? (int)cluster_rank() : 0;
+    const int cid = blockIdx.x / g.G;
+    int b, seg;
+    if constexpr (RECOMPUTE) {
+        b = cid / a.J;
+        seg = cid % a.J;
+    } else {
+        b = cid;
+        seg = 0;
+    }
+    const int L = a.lengths[b];
+    if (L < 1 || L > a.T) {
+        if (rank == 0 && tid == 0 && seg == 0) set_status(a.status, SEMICRF_ERR_INVALID_LENGTH);
+        return;
+    }
+    const int t0 = seg * a.delta;
+    if (RECOMPUTE && t0 >= L) return;
+    const int t_end = RECOMPUTE ? min(t0 + a.delta, L) : L;
+    const int c0l = rank * Cg, cg_own = min(Cg, C - c0l);
+    ClSmem sm = cl_smem(smc, K, C, g, false);
+    const size_t rowbase = (size_t)b * (a.T + 1);
+    unsigned char *ck_base = a.ckpt + ((size_t)b * a.J) * a.ckpt_stride;
+    int kZ = 0;
+    double cz = 0.0;
+    if constexpr (RECOMPUTE) {
+        kZ = a.lz[b].k;
+        cz = exp(-a.lz[b].logn);
+    }
+    const Roles ro = cl_roles(g, warp, lane, c0l, cg_own);
+    const int lc = ro.lc, j = ro.j, c = ro.c;
+    const bool own = ro.is_own && ro.lab_ok;
+
+    // ------------------------------------------------------------------ init
+    {
+        const unsigned char *ck = ck_base + (size_t)seg * a.ckpt_stride;
+        const double *ck_ring = reinterpret_cast<const double *>(ck);
+        double *ck_ring_w = reinterpret_cast<double *>(ck_base);
+        for (int i = tid; i < K * Cg; i += NT) {
+            const int sl = i / Cg, l2 = i % Cg;
+            const bool ok = l2 < cg_own;
+            sm.Wd[sl * RS + l2] = ok ? exp((double)a.D[(size_t)sl * C + c0l + l2]) : 0.0;
+            double v;
+            if constexpr (RECOMPUTE) {
+                v = ok ? ck_ring[(size_t)sl * C + c0l + l2] : 0.0;
+            } else {
+                v = (ok && sl == 0) ? 1.0 : 0.0;   // row 0 = exp(0), rows < 0 empty
+                if (ok) ck_ring_w[(size_t)sl * C + c0l + l2] = v;   // checkpoint 0
+            }
+            sm.ring[sl * RS + l2] = v;
+            sm.ring[(sl + K) * RS + l2] = v;
+        }
+        for (int i = tid; i < 2 * C; i += NT) sm.gath[i] = 0.0;
+        for (int i = tid; i < 4 * Cg * PW; i += NT) sm.pre3[i] = 0.0;
+        for (int i = tid; i < 2 * Cg; i += NT) sm.hbuf[i] = 0;
+        if (tid == 0) {
+            if constexpr (RECOMPUTE) {
+                const int32_t *ck_r = reinterpret_cast<const int32_t *>(ck_ring + (size_t)K * C);
+                sm.kbuf[0] = ck_r[C];       // k_{t0+1}
+                sm.kbuf[1] = ck_r[C + 1];   // k_{t0+2}
+            } else {
+                sm.kbuf[0] = 0;
+                sm.kbuf[1] = 0;
+                int32_t *ck_r = reinterpret_cast<int32_t *>(ck_ring_w + (size_t)K * C);
+                if (rank == 0) {
+                    ck_r[C] = 0;
+                    ck_r[C + 1] = 0;
+                }
+            }
+            if constexpr (CLUSTER) {
+                mbar_init(&sm.full[0], 1);
+                mbar_init(&sm.full[1], 1);
+                asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+            }
+        }
+        if (!RECOMPUTE && tid < cg_own) {
+            int32_t *ck_r = reinterpret_cast<int32_t *>(ck_ring_w + (size_t)K * C);
+            ck_r[c0l + tid] = 0;
+        }
+    }
+    __syncthreads();
+    // window sums for the first two positions, from the restored ring (one reference)
+    if (ro.is_win) {
+        for (int q = 1; q <= 2; ++q) {
+            const int tau = t0 + q;
+            const double v = ro.lab_ok ? window_fwd(sm.ring, sm.Wd, K, RS, lc, g.LPW, j, tau % K, 0) : 0.0;
+            const double s = group_sum(v, g.LPW < 32 ? g.LPW : 32);
+            if (ro.lab_ok && (j & 31) == 0) sm.pre3[(q - 1) * Cg * PW + lc * PW + (j >> 5)] = s;
+        }
+    }
+    // One register array holds either the transition weights E (transition lanes)
+    // or the chain state (owner lanes): a thread has one role, and sharing keeps
+    // the register count of the kernel that of the larger of the two.
+    // Chain state at the start of step t: U1 = U[t-1], U2 = U[t-2] (reference of
+    // t-1) and the values prepared for t from everything but U[t-1]:
+    //   pre = U[t-2] W1 + pre3_t,  e = exp(S_t + ln2 (r - k_t)),  f = exp(ln2 (k_t - r) - S_t),
+    //   pe = pre e,  w0e = W0 e,  so a'[t] = U[t-1] w0e + pe is one FMA after U[t-1].
+    constexpr int NU = CPL > 10 ? CPL : 10;
+    double R[NU];
+#pragma unroll
+    for (int m = 0; m < NU; ++m) {
+        const int cp = j + m * g.LPL;
+        R[m] = (m < CPL && ro.is_tr && ro.lab_ok && cp < C) ? exp((double)a.A[(size_t)cp * C + c]) : 0.0;
+    }
+    double(&E)[CPL] = *reinterpret_cast<double(*)[CPL]>(&R[0]);
+    double &W0 = R[0], &W1 = R[1], &U1 = R[2], &U2 = R[3], &pre = R[4], &f = R[5], &pe = R[6], &w0e = R[7],
+           &ap = R[8];
+    double f_n = 0.0;
+    int r = 0, h1 = 0, h2 = 0, kt = 0, kt_n = 0;
+    auto prefetch = [&](int tp) {
+        if (tp <= t_end) {
+            const size_t ix = (rowbase + tp) * C + c;
+            const int sl = tp & (kPF - 1);
+            cp_async8(&sm.pf_es[sl * Cg + lc], a.tES + ix);
+            cp_async8(&sm.pf_ies[sl * Cg + lc], a.tIES + ix);
+            cp_async4(&sm.pf_m[sl * Cg + lc], a.tM + ix);
+        }
+        cp_async_commit();
+    };
+    // values for position tn (step un) from row d2 = U[tn-2] at the current reference
+    auto prepare = [&](int tn, int un, double d2, double &pre_o, double &f_o, double &pe_o, double &w0e_o,
+                       int &kt_o) {
+        const int sl = tn & (kPF - 1);
+        const double es = sm.pf_es[sl * Cg + lc], ies = sm.pf_ies[sl * Cg + lc];
+        const int m = sm.pf_m[sl * Cg + lc];
+        kt_o = sm.kbuf[un & 3];
+        double p3 = 0.0;
+        for (int q = 0; q < PW; ++q) p3 += sm.pre3[(un & 3) * Cg * PW + lc * PW + q];
+        pre_o = fma(d2, W1, rescale(p3, h1 + h2));
+        const double e = es * pow2c(m + r - kt_o);   // exp(S + ln2 (r - k))
+        f_o = ies * pow2c(kt_o - r - m);             // exp(ln2 (k - r) - S)
+        pe_o = pre_o * e;
+        w0e_o = W0 * e;
+    };
+    if (own) {
+        W0 = sm.Wd[lc];
+        W1 = K >= 2 ? sm.Wd[RS + lc] : 0.0;
+        U1 = sm.ring[(t0 % K) * RS + lc];
+        U2 = K >= 2 ? sm.ring[(((t0 - 1) % K + K) % K) * RS + lc] : 0.0;
+        if constexpr (RECOMPUTE) {
+            const int32_t *ck_r = reinterpret_cast<const int32_t *>(
+                reinterpret_cast<const double *>(ck_base + (size_t)seg * a.ckpt_stride) + (size_t)K * C);
+            r = ck_r[c];
+        }
+        for (int i = 1; i < kPF; ++i) prefetch(t0 + i);
+    }
+    __syncthreads();   // look-ahead sums written
+    if (own) {
+        cp_async_wait<kPF - 2>();   // position t0+1 has landed
+        prepare(t0 + 1, 0, U2, pre, f, pe, w0e, kt);
+    }
+    if constexpr (CLUSTER) cluster_barrier();   // mbarriers of every CTA initialised
+    else __syncthreads();
+
+    int tK = (t0 + 1) % K;
+    int td = (t0 + 1) % a.delta;
+    bool timed_out = false;
+    for (int t = t0 + 1; t <= t_end; ++t) {
+        const int u = t - t0 - 1;   // step count
+        const int par = u & 1;
+        if (ro.is_own) {
+            // ------------------------------------------------ owners: chain
+            if (own) {
+                ap = fma(U1, w0e, pe);
+                if constexpr (CLUSTER) {
+                    for (int g2 = 0; g2 < g.G; ++g2) st_async_f64(&sm.gath[par * C + c], &sm.full[par], g2, ap);
+                } else {
+                    sm.gath[par * C + c] = ap;
+                }
+                // rebase when p = a' / e leaves [2^-512, 2^512]
+                const double p = fma(U1, W0, pre);
+                const int ex = exponent_of(p);
+                const int h = (ex > kRebaseBits || ex < -kRebaseBits) ? -ex : 0;
+                if (h != 0) {
+                    const double s2 = pow2(h);
+                    r -= h;
+                    f *= s2;
+                    U1 *= s2;
+                }
+                sm.hbuf[par * Cg + lc] = h;
+                h2 = h1;
+                h1 = h;
+                // prepare position t+1 (row t-1 = U1 is its d = 2 row)
+                prefetch(t + kPF - 1);     // into the slot position t-1 used
+                cp_async_wait<kPF - 2>();  // position t+1 has landed
+                if (t < t_end) prepare(t + 1, u + 1, U1, pre, f_n, pe, w0e, kt_n);
+            }
+            if constexpr (!CLUSTER) {
+                cta_arrive(1, NOT);   // a'[t] stored (for the transition warps)
+                if (g.NWO > 1) cta_barrier(7, 32 * g.NWO);
+                else __syncwarp();
+            }
+            if (warp == 0) {
+                // normaliser n_t = sum_c a'[t,c] (the same in every CTA)
+                if (!wait_values<CLUSTER>(sm, par, u, timed_out)) {
+                    timed_out = true;
+                    set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
+                }
+                const double n = warp_total(sm.gath + par * C, C, lane);
+                if (lane == 0) {
+                    const int kk = sm.kbuf[u & 3];
+                    if (t == L) {
+                        if (!RECOMPUTE && rank == 0) {
+                            const double lz = kLn2 * (double)kk + log(n);
+                            a.logZ[b] = lz;
+                            a.lz[b].logn = log(n);
+                            a.lz[b].k = kk;
+                            if (!isfinite(lz)) set_status(a.status, SEMICRF_ERR_DEVICE_RANGE);
+                        }
+                    } else {
+                        sm.kbuf[(u + 2) & 3] = kk + exponent_of(n);
+                    }
+                }
+            }
+            cta_barrier(4, NOT);   // q[t] ready
+            // ------------------------------------------------ owners: new row
+            if (own) {
+                const size_t row = (rowbase + t) * C + c;
+                if (t < L) {
+                    const double U = sm.qbuf[lc] * f;
+                    sm.ring[tK * RS + lc] = U;
+                    sm.ring[(tK + K) * RS + lc] = U;
+                    U2 = U1;
+                    U1 = U;
+                    if constexpr (RECOMPUTE) {
+                        a.cU[row] = U * cz;
+                        a.cA[row] = ap * cz;
+                        a.eU[row] = r - kZ;
+                    }
+                } else if constexpr (RECOMPUTE) {
+                    a.cA[row] = ap * cz;
+                }
+                if (RECOMPUTE && c == 0) a.eA[rowbase + t] = kt - kZ;
+                f = f_n;
+                kt = kt_n;
+            }
+        } else if (ro.is_tr) {
+            // -------------------------------------------------------- transition
+            if constexpr (CLUSTER) {
+                if (!wait_values<CLUSTER>(sm, par, u, timed_out)) {
+                    timed_out = true;
+                    set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
+                }
+            } else {
+                cta_barrier(1, NOT);
+            }
+            double v[CPL];
+#pragma unroll
+            for (int m = 0; m < CPL; ++m) {
+                const int cp = j + m * g.LPL;
+                v[m] = cp < C ? sm.gath[par * C + cp] : 0.0;
+            }
+            const double q = group_sum(tree_dot<CPL>(v, E), g.LPL);
+            if (ro.lab_ok && j == 0) sm.qbuf[lc] = q;
+            cta_arrive(4, NOT);
+        } else if (ro.is_win) {
+            // ------------------------------------- window sums two positions ahead
+            if (CLUSTER && tid == W0T) mbar_expect_tx(&sm.full[par], C * 8);
+            const int hp = ro.lab_ok ? sm.hbuf[(par ^ 1) * Cg + lc] : 0;   // rebase at t-1
+            const int tau2K = (tK + 2) % K;
+            const double v = ro.lab_ok ? window_fwd(sm.ring, sm.Wd, K, RS, lc, g.LPW, j, tau2K, hp) : 0.0;
+            const double s = group_sum(v, g.LPW < 32 ? g.LPW : 32);
+            if (ro.lab_ok && (j & 31) == 0) sm.pre3[((u + 2) & 3) * Cg * PW + lc * PW + (j >> 5)] = s;
+        }
+        if (cta_barrier_or(2, NT, timed_out)) timed_out = true;
+        if (!RECOMPUTE && td == 0 && t < L) {
+            // checkpoint t / delta: the ring at the reference of position t, r, k_{t+1}, k_{t+2}.
+            // Row age 0 (row t) is there; ages 1..K-2 are at the reference of t-1; the
+            // oldest row (age K-1, K >= 3) at that of t-2.
+            unsigned char *ck = ck_base + (size_t)(t / a.delta) * a.ckpt_stride;
+            double *ck_ring = reinterpret_cast<double *>(ck);
+            int32_t *ck_r = reinterpret_cast<int32_t *>(ck_ring + (size_t)K * C);
+            for (int i = tid; i < K * Cg; i += NT) {
+                const int sl = i / Cg, l2 = i % Cg;
+                if (l2 < cg_own) {
+                    int age = tK - sl;
+                    if (age < 0) age += K;
+                    int hh = 0;
+                    if (age >= 1) hh = sm.hbuf[par * Cg + l2];
+                    if (age == K - 1 && K >= 3) hh += sm.hbuf[(par ^ 1) * Cg + l2];
+                    ck_ring[(size_t)sl * C + c0l + l2] = rescale(sm.ring[sl * RS + l2], hh);
+                }
+            }
+            if (own) ck_r[c] = r;
+            if (rank == 0 && tid == 0) {
+                ck_r[C] = sm.kbuf[(u + 1) & 3];
+                ck_r[C + 1] = sm.kbuf[(u + 2) & 3];
+            }
+            cta_barrier(3, NT);
+        }
+        tK = (tK + 1 == K) ? 0 : tK + 1;
+        td = (td + 1 == a.delta) ? 0 : td + 1;
+    }
+    if constexpr (CLUSTER) cluster_barrier();   // no CTA leaves while peers may still store to it
+}
+
+template <int CPL, int MAXT, bool CLUSTER>
+__global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
+{
+    extern __shared__ __align__(16) double smc[];
+    const int K = a.K, C = a.C, Cg = g.Cg, NT = g.NT, RS = g.RS, PW = g.PW;
+    const int NOT = 32 * (g.NWO + g.NWT);
+    const int W0T = 32 * (g.NWO + g.NWT);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rank = CLUSTER ? (int)cluster_rank() : 0;
+    const int b = blockIdx.x / g.G;
+    const int L = a.lengths[b];
+    if (L < 1 || L > a.T) {
+        if (rank == 0 && tid == 0) set_status(a.status, SEMICRF_ERR_INVALID_LENGTH);
+        return;
+    }
+    const int c0l = rank * Cg, cg_own = min(Cg, C - c0l);
+    ClSmem sm = cl_smem(smc, K, C, g, true);
+    const size_t rowbase = (size_t)b * (a.T + 1);
+    const int kZ = a.lz[b].k;
+    const double cz = exp(-a.lz[b].logn);
+    const Roles ro = cl_roles(g, warp, lane, c0l, cg_own);
+    const int lc = ro.lc, j = ro.j, c = ro.c;
+    const bool own = ro.is_own && ro.lab_ok;
+
+    // ------------------------------------------------------------------ init
+    // row L: be = 0, so V[L,c] = exp(S[L,c] - ln2 rb) = es with rb = m; rows > L empty
+    for (int i = tid; i < K * Cg; i += NT) {
+        const int sl = i / Cg, l2 = i % Cg;
+        const bool ok = l2 < cg_own;
+        sm.Wd[sl * RS + l2] = ok ? exp((double)a.D[(size_t)sl * C + c0l + l2]) : 0.0;
+        const size_t ixL = (rowbase + L) * C + c0l + l2;
+        const double v = (ok && sl == L % K) ? a.tES[ixL] : 0.0;
+        sm.ring[sl * RS + l2] = v;
+        sm.ring[(sl + K) * RS + l2] = v;
+    }
+    for (int i = tid; i < 2 * C; i += NT) sm.gath[i] = 0.0;
+    for (int i = tid; i < 4 * Cg * PW; i += NT) sm.pre3[i] = 0.0;   // positions L-1, L-2: no rows beyond L
+    for (int i = tid; i < 2 * Cg; i += NT) sm.hbuf[i] = 0;
+    if (tid == 0) {
+        sm.kbuf[0] = 0;
+        sm.kbuf[1] = 0;
+        if constexpr (CLUSTER) {
+            mbar_init(&sm.full[0], 1);
+            mbar_init(&sm.full[1], 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+    }
+    // One register array holds either the transposed transition weights Er
+    // (transition lanes) or the chain state (owner lanes).
+    // Chain state at the start of step s: V1 = V[s+1], V2 = V[s+2] (reference of
+    // s+1) and, prepared from everything but V[s+1]:
+    //   pre = V[s+2] W1 + pre3_s, eb = exp(ln2 (rb - kb) - S_s), gg = exp(S_s + ln2 (kb - rb)),
+    //   pbe = pre eb, w0e = W0 eb, so bp[s] = V[s+1] w0e + pbe is one FMA after V[s+1];
+    //   coef = X[s] (start factor at the reference rb), a2 (transition factor).
+    constexpr int NU = CPL > 14 ? CPL : 14;
+    double R[NU];
+#pragma unroll
+    for (int m = 0; m < NU; ++m) {
+        const int cc = j + m * g.LPL;
+        R[m] = (m < CPL && ro.is_tr && ro.lab_ok && cc < C) ? exp((double)a.A[(size_t)c * C + cc]) : 0.0;
+    }
+    double(&Er)[CPL] = *reinterpret_cast<double(*)[CPL]>(&R[0]);
+    double &W0 = R[0], &W1 = R[1], &V1 = R[2], &V2 = R[3], &pre = R[4], &gg = R[5], &pbe = R[6], &w0e = R[7],
+           &coef = R[8], &a2 = R[9], &mu_acc = R[10], &musum = R[11], &bp = R[12], &start = R[13];
+    double gg_n = 0.0, coef_n = 0.0, a2_n = 0.0;
+    int rb = 0, h1 = 0, h2 = 0, kb = 0, kb_n = 0;
+    auto prefetch = [&](int sp) {   // owners: position sp's tables and recomputed rows
+        if (sp >= 0) {
+            const size_t ix = (rowbase + sp) * C + c;
+            const int sl = sp & (kPF - 1);
+            cp_async8(&sm.pf_es[sl * Cg + lc], a.tES + ix);
+            cp_async8(&sm.pf_ies[sl * Cg + lc], a.tIES + ix);
+            cp_async4(&sm.pf_m[sl * Cg + lc], a.tM + ix);
+            if (sp >= 1) {
+                cp_async8(&sm.pf_cu[sl * Cg + lc], a.cU + ix);
+                cp_async8(&sm.pf_ca[sl * Cg + lc], a.cA + ix);
+                cp_async4(&sm.pf_eu[sl * Cg + lc], a.eU + ix);
+                cp_async4(&sm.pf_ea[sl * Cg + lc], a.eA + rowbase + sp);
+            }
+        }
+        cp_async_commit();
+    };
+    auto prepare = [&](int sn, int un, double d2, double &pre_o, double &gg_o, double &pbe_o, double &w0e_o,
+                       double &coef_o, double &a2_o, int &kb_o) {
+        const int sl = sn & (kPF - 1);
+        kb_o = sm.kbuf[un & 3];
+        double p3 = 0.0;
+        for (int q = 0; q < PW; ++q) p3 += sm.pre3[(un & 3) * Cg * PW + lc * PW + q];
+        pre_o = fma(d2, W1, rescale(p3, h1 + h2));
+        const int m = sm.pf_m[sl * Cg + lc];
+        gg_o = sm.pf_es[sl * Cg + lc] * pow2c(m + kb_o - rb);               // exp(S + ln2 (kb - rb))
+        const double eb = sm.pf_ies[sl * Cg + lc] * pow2c(rb - kb_o - m);   // exp(ln2 (rb - kb) - S)
+        pbe_o = pre_o * eb;
+        w0e_o = W0 * eb;
+        coef_o = (sn == 0) ? scale2c(cz, rb - kZ) : scale2c(sm.pf_cu[sl * Cg + lc], sm.pf_eu[sl * Cg + lc] + rb);
+        a2_o = (sn >= 1) ? scale2c(sm.pf_ca[sl * Cg + lc], sm.pf_ea[sl * Cg + lc] + kb_o) : 0.0;
+    };
+    if (own) {
+        W0 = exp((double)a.D[c]);
+        W1 = K >= 2 ? exp((double)a.D[C + c]) : 0.0;
+        V2 = 0.0;
+        musum = 0.0;
+        rb = a.tM[(rowbase + L) * C + c];
+        V1 = a.tES[(rowbase + L) * C + c];
+        a.Vst[(rowbase + L) * C + c] = V1;
+        a.rbst[(rowbase + L) * C + c] = rb;
+        mu_acc = scale2(a.cA[(rowbase + L) * C + c], a.eA[rowbase + L]);
+        for (int i = 1; i < kPF; ++i) prefetch(L - i);
+        cp_async_wait<kPF - 2>();   // position L-1 has landed
+        prepare(L - 1, 0, V2, pre, gg, pbe, w0e, coef, a2, kb);
+    }
+    if constexpr (CLUSTER) cluster_barrier();
+    else __syncthreads();
+
+    int sK = (L - 1) % K;   // s mod K
+    bool timed_out = false;
+    for (int s = L - 1; s >= 0; --s) {
+        const int u = L - 1 - s;   // step count: buffers by u
+        const int par = u & 1;
+        if (ro.is_own) {
+            // ------------------------------------------------ owners: chain
+            if (own) {
+                bp = fma(V1, w0e, pbe);
+                if constexpr (CLUSTER) {
+                    for (int g2 = 0; g2 < g.G; ++g2) st_async_f64(&sm.gath[par * C + c], &sm.full[par], g2, bp);
+                } else {
+                    sm.gath[par * C + c] = bp;
+                }
+                const double pb = fma(V1, W0, pre);
+                start = coef * pb;   // marginal of a segment of label c starting at s
+                const int ex = exponent_of(pb);
+                const int h = (ex > kRebaseBits || ex < -kRebaseBits) ? -ex : 0;
+                if (h != 0) {
+                    const double s2 = pow2(h);
+                    rb -= h;
+                    gg *= s2;
+                    V1 *= s2;
+                }
+                sm.hbuf[par * Cg + lc] = h;
+                h2 = h1;
+                h1 = h;
+                prefetch(s - (kPF - 1));    // into the slot position s+1 used
+                cp_async_wait<kPF - 2>();   // position s-1 has landed
+                if (s >= 1) prepare(s - 1, u + 1, V1, pre, gg_n, pbe, w0e, coef_n, a2_n, kb_n);
+            }
+            if constexpr (!CLUSTER) {
+                cta_arrive(1, NOT);
+                if (g.NWO > 1) cta_barrier(7, 32 * g.NWO);
+                else __syncwarp();
+            }
+            if (warp == 0) {
+                // backward normaliser (the same in every CTA)
+                if (!wait_values<CLUSTER>(sm, par, u, timed_out)) {
+                    timed_out = true;
+                    set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
+                }
+                const double n = warp_total(sm.gath + par * C, C, lane);
+                if (lane == 0) {
+                    const int kk = sm.kbuf[u & 3];
+                    if (s == 0) {
+                        if (rank == 0) a.logzb[b] = kLn2 * (double)kk + log(n);
+                    } else if (s >= 2) {
+                        sm.kbuf[(u + 2) & 3] = kk + exponent_of(n);
+                    }
+                }
+            }
+            cta_barrier(4, NOT);
+            // ------------------------------------------------ owners: new row
+            if (own) {
+                // mu_acc holds the coverage of x[s] by label c; moving to x[s-1] adds the
+                // segments ending at s and removes those starting at s
+                const size_t row = (rowbase + s) * C + c;
+                a.dX[((size_t)b * a.T + s) * C + c] = (float)mu_acc;
+                musum += mu_acc;
+                if (s >= 1) {
+                    const double q = sm.qbuf[lc];
+                    const double V = q * gg;
+                    sm.ring[sK * RS + lc] = V;
+                    sm.ring[(sK + K) * RS + lc] = V;
+                    V2 = V1;
+                    V1 = V;
+                    mu_acc += a2 * q - start;
+                    a.Vst[row] = V;
+                    a.rbst[row] = rb;
+                    a.bpst[row] = bp;
+                    if (c == 0) a.kbst[rowbase + s] = kb;
+                } else {
+                    mu_acc -= start;
+                }
+                gg = gg_n;
+                coef = coef_n;
+                a2 = a2_n;
+                kb = kb_n;
+            }
+        } else if (ro.is_tr) {
+            // ------------------------------------------- transposed transition
+            if constexpr (CLUSTER) {
+                if (!wait_values<CLUSTER>(sm, par, u, timed_out)) {
+                    timed_out = true;
+                    set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
+                }
+            } else {
+                cta_barrier(1, NOT);
+            }
+            double v[CPL];
+#pragma unroll
+            for (int m = 0; m < CPL; ++m) {
+                const int cc = j + m * g.LPL;
+                v[m] = cc < C ? sm.gath[par * C + cc] : 0.0;
+            }
+            const double q = group_sum(tree_dot<CPL>(Er, v), g.LPL);
+            if (ro.lab_ok && j == 0) sm.qbuf[lc] = q;
+            cta_arrive(4, NOT);
+        } else if (ro.is_win) {
+            // ----------------------- window sums two positions ahead (position s-2)
+            if (CLUSTER && tid == W0T) mbar_expect_tx(&sm.full[par], C * 8);
+            const int hp = ro.lab_ok ? sm.hbuf[(par ^ 1) * Cg + lc] : 0;   // rebase at s+1
+            const double v = ro.lab_ok ? window_bwd(sm.ring, sm.Wd, K, RS, lc, g.LPW, j, sK, hp) : 0.0;
+            const double sum = group_sum(v, g.LPW < 32 ? g.LPW : 32);
+            if (ro.lab_ok && (j & 31) == 0 && s >= 2) sm.pre3[((u + 2) & 3) * Cg * PW + lc * PW + (j >> 5)] = sum;
+        }
+        if (cta_barrier_or(2, NT, timed_out)) timed_out = true;
+        sK = (sK == 0) ? K - 1 : sK - 1;
+    }
+    if (own) {
+        a.musum[(size_t)b * C + c] = musum;
+        a.mures[(size_t)b * C + c] = mu_acc;
+    }
+    if constexpr (CLUSTER) cluster_barrier();
+}
+
+template <int CPL, int MAXT>
+cudaError_t launch_cl_bwd_tpl(const ClGeom &g, const FbArgs &a, cudaStream_t st)
+{
+    const bool cl = g.G > 1;
+    void *fn = cl ? (void *)cl_bwd_kernel<CPL, MAXT, true> : (void *)cl_bwd_kernel<CPL, MAXT, false>;
+    const size_t smem = cl_smem_bytes_impl(a.K, a.C, g, true);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (g.G > 8) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)a.B * g.G);
+    cfg.blockDim = dim3(g.NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (cl) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = g.G;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    FbArgs aa = a;
+    ClGeom gg = g;
+    void *args[] = {&aa, &gg};
+    prof_before(st);
+    e = cudaLaunchKernelExC(&cfg, fn, args);
+    prof_after(st);
+    return e;
+}
+
+template <int CPL, int MAXT>
+cudaError_t launch_cl_fwd_tpl(const ClGeom &g, const FbArgs &a, cudaStream_t st, bool recompute)
+{
+    const bool cl = g.G > 1;
+    void *fn = recompute ? (cl ? (void *)cl_fwd_kernel<CPL, MAXT, true, true> : (void *)cl_fwd_kernel<CPL, MAXT, false, true>)
+                         : (cl ? (void *)cl_fwd_kernel<CPL, MAXT, true, false> : (void *)cl_fwd_kernel<CPL, MAXT, false, false>);
+    const size_t smem = cl_smem_bytes_impl(a.K, a.C, g, false);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (g.G > 8) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    const unsigned nclusters = recompute ? (unsigned)a.B * (unsigned)a.J : (unsigned)a.B;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nclusters * g.G);
+    cfg.blockDim = dim3(g.NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (cl) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = g.G;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    FbArgs aa = a;
+    ClGeom gg = g;
+    void *args[] = {&aa, &gg};
+    prof_before(st);
+    e = cudaLaunchKernelExC(&cfg, fn, args);
+    prof_after(st);
+    return e;
+}
+
+int cl_max_threads(int nt) { return nt <= 256 ? 256 : nt <= 512 ? 512 : nt <= 768 ? 768 : 1024; }
+int cl_cpl_bucket(int cpl) { return cpl <= 4 ? 4 : cpl <= 8 ? 8 : cpl <= 16 ? 16 : 32; }
+
+int pow2_floor(int v)
+{
+    int p = 1;
+    while (p * 2 <= v) p *= 2;
+    return p;
+}
+
+int pow2_ceil(int v)
+{
+    int p = 1;
+    while (p < v) p *= 2;
+    return p;
+}
+
+}  // namespace
+
+// One candidate geometry: G CTAs, LPL transition lanes per label, LPW window
+// lanes per label.  Returns false when it does not fit 1024 threads or shared
+// memory.  *cost estimates the cycles of one position from the latencies of
+// this part (a dependent FP64 operation ~33 cycles, a shared load ~55, a shuffle
+// level with its add ~58, the cluster exchange ~230): the owner-transition
+// chain and the window warps run in parallel, the slower one sets the pace.
+// Register classes that spill (more than 512 threads, or 32 transition terms
+// per lane with more than 256) pay extra.
+static bool cl_try(int K, int C, bool bwd, int G, int LPL, int LPW, ClGeom *out, double *cost)
+{
+    ClGeom g;
+    g.G = G;
+    if (G > C) return false;
+    g.Cg = (C + G - 1) / G;
+    if ((G - 1) * g.Cg >= C) return false;   // every CTA owns at least one label
+    g.RS = g.Cg | 1;
+    g.LPL = LPL;
+    if (LPL < 1 || LPL > 32 || (LPL & (LPL - 1))) return false;
+    g.CPL = (C + LPL - 1) / LPL;
+    if (g.CPL > 32) return false;
+    g.NWO = (g.Cg + 31) / 32;
+    g.NWT = (g.Cg * LPL + 31) / 32;
+    const int rows = K > 2 ? K - 2 : 1;   // window rows d = 3..K (forward), i = 1..K-2 (backward)
+    g.LPW = LPW;
+    if (LPW < 1 || LPW > 256 || (LPW & (LPW - 1)) || LPW > rows) return false;
+    g.PW = g.LPW > 32 ? g.LPW / 32 : 1;
+    g.NWW = (g.Cg * g.LPW + 31) / 32;
+    if (g.NWW < 1) g.NWW = 1;
+    g.NT = 32 * (g.NWO + g.NWT + g.NWW);
+    if (g.NT > 1024) return false;
+    const int maxt = cl_max_threads(g.NT);
+    const int cpl = cl_cpl_bucket(g.CPL);
+    if (cpl == 32 && maxt > 512) return false;
+    if (cpl == 16 && maxt > 768) return false;
+    const size_t smem = cl_smem_bytes_impl(K, C, g, bwd);
+    if (smem > kSmemBudget) return false;
+    auto lg2 = [](int v) {
+        int l = 0;
+        while ((1 << l) < v) ++l;
+        return l;
+    };
+    const int R = (rows + LPW - 1) / LPW;
+    const double chain = 33 + (G > 1 ? 230 + 10 * G : 40) + 55 + 33 * (1 + lg2(cpl)) + 58 * lg2(LPL) + 150;
+    const double window = ((R + 7) / 8) * 190.0 + 58 * lg2(LPW < 32 ? LPW : 32) + 60;
+    double c = chain > window ? chain : window;
+    if (maxt > 512 || (cpl == 32 && maxt > 256)) c += 400;   // register classes that spill
+    *out = g;
+    *cost = c;
+    return true;
+}
+
+// The cheapest geometry by the cost model (ties: the smaller cluster).
+// SEMICRF_CL_PLAN="G,LPL,LPW" (0 = free choice for that field) restricts the
+// search; the shape is unsupported if nothing fits.
+bool cl_plan(int K, int C, bool bwd, ClGeom *out)
+{
+    int fG = 0, fL = 0, fW = 0;
+    const char *env = getenv("SEMICRF_CL_PLAN");
+    if (env && *env && sscanf(env, "%d,%d,%d", &fG, &fL, &fW) < 1) return false;
+    bool found = false;
+    double best = 0.0;
+    for (int G = 1; G <= 16; G *= 2) {
+        if (fG > 0 && G != fG) continue;
+        for (int LPL = 1; LPL <= 32; LPL *= 2) {
+            if (fL > 0 && LPL != fL) continue;
+            for (int LPW = 1; LPW <= 256; LPW *= 2) {
+                if (fW > 0 && LPW != fW) continue;
+                ClGeom g;
+                double cost;
+                if (!cl_try(K, C, bwd, G, LPL, LPW, &g, &cost)) continue;
+                if (!found || cost < best) {
+                    best = cost;
+                    *out = g;
+                    found = true;
+                }
+            }
+        }
+    }
+    return found;
+}
+
+#define SEMICRF_CL_CASE(CPL, MAXT, CALL) \
+    if (cpl == CPL && maxt == MAXT) return CALL<CPL, MAXT>
+#define SEMICRF_CL_TABLE(CALL, ...)                                                                        \
+    SEMICRF_CL_CASE(4, 256, CALL)(__VA_ARGS__); SEMICRF_CL_CASE(4, 512, CALL)(__VA_ARGS__);                \
+    SEMICRF_CL_CASE(4, 768, CALL)(__VA_ARGS__); SEMICRF_CL_CASE(4, 1024, CALL)(__VA_ARGS__);               \
+    SEMICRF_CL_CASE(8, 256, CALL)(__VA_ARGS__); SEMICRF_CL_CASE(8, 512, CALL)(__VA_ARGS__);                \
+    SEMICRF_CL_CASE(8, 768, CALL)(__VA_ARGS__); SEMICRF_CL_CASE(8, 1024, CALL)(__VA_ARGS__);               \
+    SEMICRF_CL_CASE(16, 256, CALL)(__VA_ARGS__); SEMICRF_CL_CASE(16, 512, CALL)(__VA_ARGS__);              \
+    SEMICRF_CL_CASE(16, 768, CALL)(__VA_ARGS__); SEMICRF_CL_CASE(32, 256, CALL)(__VA_ARGS__);              \
+    SEMICRF_CL_CASE(32, 512, CALL)(__VA_ARGS__);
+
+cudaError_t launch_cl_forward(const FbArgs &a, cudaStream_t st, bool recompute)
+{
+    ClGeom g;
+    if (!cl_plan(a.K, a.C, false, &g)) return cudaErrorInvalidConfiguration;
+    const int cpl = cl_cpl_bucket(g.CPL), maxt = cl_max_threads(g.NT);
+    SEMICRF_CL_TABLE(launch_cl_fwd_tpl, g, a, st, recompute)
+    return cudaErrorInvalidConfiguration;
+}
+
+cudaError_t launch_cl_backward(const FbArgs &a, cudaStream_t st)
+{
+    ClGeom g;
+    if (!cl_plan(a.K, a.C, true, &g)) return cudaErrorInvalidConfiguration;
+    const int cpl = cl_cpl_bucket(g.CPL), maxt = cl_max_threads(g.NT);
+    SEMICRF_CL_TABLE(launch_cl_bwd_tpl, g, a, st)
+    return cudaErrorInvalidConfiguration;
+}
+#undef SEMICRF_CL_TABLE
+#undef SEMICRF_CL_CASE
+
+}  // namespace semicrf

@@ -107,7 +107,7 @@ bool make_layout(const semicrf_dims &d, int what, const Plan &p, Layout *out)
     L.scan = take(B * L.NCH * C * 8);
     if (what == SEMICRF_WS_TRAIN) {
         L.logz = take(B * sizeof(LogZState));
-        L.ckpt_stride = align_up(K * C * 8 + (C + 1) * 4, 256);
+        L.ckpt_stride = align_up(K * C * 8 + (C + 2) * 4, 256);
         L.ckpt = take(B * (size_t)L.J * L.ckpt_stride);
         L.tES = take(B * (T + 1) * C * 8);
         L.tIES = take(B * (T + 1) * C * 8);
@@ -118,6 +118,13 @@ bool make_layout(const semicrf_dims &d, int what, const Plan &p, Layout *out)
         L.eA = take(B * (T + 1) * 4);
         L.accD = take(B * K * C * 8);
         L.accA = take(B * C * C * 8);
+        L.Vst = take(B * (T + 1) * C * 8);
+        L.rbst = take(B * (T + 1) * C * 4);
+        L.bpst = take(B * (T + 1) * C * 8);
+        L.kbst = take(B * (T + 1) * 4);
+        cl_grad_splits(d.B, d.T, d.K, d.C, &L.nsD, &L.nsA);
+        L.partD = take((size_t)L.nsD * K * C * 8);
+        L.partA = take((size_t)L.nsA * C * C * 8);
         L.musum = take(B * C * 8);
         L.mures = take(B * C * 8);
         L.logzb = take(B * 8);
@@ -146,7 +153,12 @@ semicrf_status check_dims_impl(const semicrf_dims *d)
         return SEMICRF_ERR_INVALID_ARG;
     if (d->C > SEMICRF_MAX_C || d->K > SEMICRF_MAX_K) return SEMICRF_ERR_UNSUPPORTED_SHAPE;
     if ((long long)d->B * (d->T + 1) * d->C > (1LL << 40)) return SEMICRF_ERR_UNSUPPORTED_SHAPE;
-    if (!make_plan(d->K, d->C).ok()) return SEMICRF_ERR_UNSUPPORTED_SHAPE;
+    if (!make_plan(d->K, d->C).ok()) return SEMICRF_ERR_UNSUPPORTED_SHAPE;   // Viterbi layout
+    if (!small_path_ok(d->K, d->C)) {
+        ClGeom g;
+        if (!cl_plan(d->K, d->C, false, &g) || !cl_plan(d->K, d->C, true, &g))
+            return SEMICRF_ERR_UNSUPPORTED_SHAPE;
+    }
     return SEMICRF_OK;
 }
 
@@ -202,6 +214,14 @@ FbArgs fb_args(const semicrf_dims *d, const Layout &lay, void *ws)
     a.musum = at<double>(ws, lay.musum);
     a.mures = at<double>(ws, lay.mures);
     a.logzb = at<double>(ws, lay.logzb);
+    a.Vst = at<double>(ws, lay.Vst);
+    a.rbst = at<int32_t>(ws, lay.rbst);
+    a.bpst = at<double>(ws, lay.bpst);
+    a.kbst = at<int32_t>(ws, lay.kbst);
+    a.nsD = lay.nsD;
+    a.nsA = lay.nsA;
+    a.partD = at<double>(ws, lay.partD);
+    a.partA = at<double>(ws, lay.partA);
     a.status = at<int32_t>(ws, lay.status);
     return a;
 }

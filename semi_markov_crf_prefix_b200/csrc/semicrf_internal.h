@@ -45,7 +45,7 @@ struct Layout {
     size_t scan = 0;        // double [B][NCH][C]
     size_t logz = 0;        // LogZState [B]
     size_t ckpt = 0;        // [B][J] records of ckpt_stride bytes
-    size_t ckpt_stride = 0; // ring double[K*C], r int32[C], k int32
+    size_t ckpt_stride = 0; // ring double[K*C], r int32[C], two normaliser exponents int32
     // Recomputed forward quantities per position t and label c, as mantissa and
     // power-of-two exponent relative to Z:
     //   exp(at[t,c] - S[t,c] - log Z) = cU * 2^eU,   exp(al[t,c] - log Z) = cA * 2^eA
@@ -59,6 +59,16 @@ struct Layout {
     size_t eA = 0;          // int32  [B][T+1]
     size_t accD = 0;        // double [B][K][C]
     size_t accA = 0;        // double [B][C][C]
+    // Cluster-kernel backward rows, consumed by the parameter-gradient kernels:
+    //   V[t,c] = exp(ga[t,c] + S[t,c] - ln2 rb[t,c]) at the reference rb it was written at,
+    //   bp[s,c] = exp(be[s,c] - ln2 kb[s]) (normalised beta), kb[s] the backward normaliser.
+    size_t Vst = 0;         // double [B][T+1][C]
+    size_t rbst = 0;        // int32  [B][T+1][C]
+    size_t bpst = 0;        // double [B][T+1][C]
+    size_t kbst = 0;        // int32  [B][T+1]
+    int nsD = 0, nsA = 0;   // partial-sum splits of the dD and dA contractions
+    size_t partD = 0;       // double [nsD][K][C]
+    size_t partA = 0;       // double [nsA][C][C]
     size_t musum = 0;       // double [B][C]
     size_t mures = 0;       // double [B][C]
     size_t logzb = 0;       // double [B]
@@ -104,10 +114,33 @@ struct FbArgs {
     double *tES, *tIES;
     int32_t *tM;
     double *accD, *accA, *musum, *mures, *logzb;
+    double *Vst, *bpst, *partD, *partA;
+    int32_t *rbst, *kbst;
+    int nsD, nsA;
     float *dX;
     double *dA, *dD;
     int32_t *status;
 };
+// Cluster kernels (fb_cluster.cu): G CTAs per sequence, Cg labels per CTA.  In a
+// CTA the first NWO warps are owner warps (one lane per label runs its chain),
+// the next NWT warps transition warps (LPL lanes per label, CPL terms per lane),
+// the next NWW warps window warps (LPW lanes per label; PW partial sums per label
+// when LPW > 32).
+// RS is the shared-memory row stride (doubles) of the ring, duration-weight and
+// duration-accumulator arrays: odd, so that the lanes of one label, which read
+// consecutive rows, fall in different banks.
+struct ClGeom {
+    int G = 0, Cg = 0, LPL = 0, CPL = 0, LPW = 0, PW = 0, NWO = 0, NWT = 0, NWW = 0, NT = 0, RS = 0;
+};
+bool cl_plan(int K, int C, bool bwd, ClGeom *out);
+cudaError_t launch_cl_forward(const FbArgs &a, cudaStream_t st, bool recompute);
+cudaError_t launch_cl_backward(const FbArgs &a, cudaStream_t st);
+// dD and dA from the cluster backward's stored rows (cl_grads.cu): two contraction
+// kernels writing split partial sums, one kernel reducing them (3 launches).
+constexpr int kGradChunk = 64;   // start positions per staged chunk
+void cl_grad_splits(int B, int T, int K, int C, int *nsD, int *nsA);
+cudaError_t launch_cl_param_grads(const FbArgs &a, cudaStream_t st);
+
 // Warp-per-sequence kernels for C <= 32, K <= 32 (kind 0 forward, 1 recompute, 2 backward).
 bool small_path_ok(int K, int C);
 cudaError_t launch_small(const FbArgs &a, cudaStream_t st, int kind);

@@ -110,6 +110,19 @@ def test_named_small_cluster_kernels(name, monkeypatch):
     check_against_oracle(w, run_gpu(w))
 
 
+@pytest.mark.parametrize("plan", ["1,0,0", "2,4,0", "4,0,1", "4,2,2", "8,0,0", "0,0,4"])
+def test_cluster_geometries(plan, monkeypatch):
+    # the cluster kernels under other splits of the labels over CTAs (G), of the
+    # transition terms over lanes (LPL) and of the window rows over lanes (LPW)
+    monkeypatch.setenv("SEMICRF_KERNEL_PATH", "general")
+    monkeypatch.setenv("SEMICRF_CL_PLAN", plan)
+    w = wl.random_small(seed=21, B=3, T=150, K=40, C=24, ragged=True)
+    check_against_oracle(w, run_gpu(w))
+    w = wl.random_small(seed=22, B=2, T=90, K=1, C=40, ragged=True)   # K = 1: duration-1 terms only
+    if plan in ("1,0,0", "2,4,0", "8,0,0"):
+        check_against_oracle(w, run_gpu(w))
+
+
 def test_kernel_families_agree():
     import os
     w = wl.make_workload("ner", B=8)
