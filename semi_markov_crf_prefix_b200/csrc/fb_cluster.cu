@@ -95,28 +95,33 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, int bytes)
                  : "memory");
 }
 
+// One potentially blocking test of the phase: the warp is suspended (not
+// spinning, so it takes no issue slots from the warps doing the work) until the
+// phase completes or about 0.5 ms pass.
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
 {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(500000u)
         : "memory");
     return done != 0;
 }
 
 // Wait (bounded) for the completion of the mbarrier phase of the given parity.
+// One warp of the CTA polls; the others block on a named barrier it arrives at.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
 {
     const uint32_t a = smem_addr(bar);
     if (mbar_try(a, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try(a, parity))
-        if (clock64() - t0 > kWaitCycles) return false;
-    return true;
+    for (unsigned i = 1;; ++i) {
+        if (mbar_try(a, parity)) return true;
+        if ((i & 63) == 0 && clock64() - t0 > kWaitCycles) return false;
+    }
 }
 
 // Store v at the address of `local` in CTA `rank` of the cluster and complete 8
@@ -320,9 +325,10 @@ __device__ __forceinline__ Roles cl_roles(const ClGeom &g, int warp, int lane, i
     return r;
 }
 
-// Waits of the transition warps and of owner warp 0 (which forms the normaliser)
-// for the C values of a position: the mbarrier of the cluster exchange, or with
-// one CTA a named barrier after the owners' plain stores.
+// Wait of owner warp 0 for the C values of a position: the mbarrier of the
+// cluster exchange (with one CTA the owners' plain stores are already ordered by
+// the barriers around this call).  Warp 0 then releases the transition warps
+// through named barrier 5, so only one warp polls.
 template <bool CLUSTER>
 __device__ __forceinline__ bool wait_values(ClSmem &sm, int par, int u, bool skip)
 {
@@ -340,6 +346,7 @@ __global__ void __launch_bounds__(MAXT, 1) cl_fwd_kernel(FbArgs a, ClGeom g)
     extern __shared__ __align__(16) double smc[];
     const int K = a.K, C = a.C, Cg = g.Cg, NT = g.NT, RS = g.RS, PW = g.PW;
     const int NOT = 32 * (g.NWO + g.NWT);   // owner + transition threads
+    const int NXW = 32 * (1 + g.NWT);       // owner warp 0 + transition threads
     const int W0T = 32 * (g.NWO + g.NWT);   // first window thread
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rank = CLUSTER ? (int)cluster_rank() : 0;
@@ -539,6 +546,7 @@ __global__ void __launch_bounds__(MAXT, 1) cl_fwd_kernel(FbArgs a, ClGeom g)
                     timed_out = true;
                     set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
                 }
+                if constexpr (CLUSTER) cta_arrive(5, NXW);   // a'[t] of every label has arrived
                 const double n = warp_total(sm.gath + par * C, C, lane);
                 if (lane == 0) {
                     const int kk = sm.kbuf[u & 3];
@@ -579,14 +587,8 @@ __global__ void __launch_bounds__(MAXT, 1) cl_fwd_kernel(FbArgs a, ClGeom g)
             }
         } else if (ro.is_tr) {
             // -------------------------------------------------------- transition
-            if constexpr (CLUSTER) {
-                if (!wait_values<CLUSTER>(sm, par, u, timed_out)) {
-                    timed_out = true;
-                    set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
-                }
-            } else {
-                cta_barrier(1, NOT);
-            }
+            if constexpr (CLUSTER) cta_barrier(5, NXW);
+            else cta_barrier(1, NOT);
             double v[CPL];
 #pragma unroll
             for (int m = 0; m < CPL; ++m) {
@@ -643,6 +645,7 @@ __global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
     extern __shared__ __align__(16) double smc[];
     const int K = a.K, C = a.C, Cg = g.Cg, NT = g.NT, RS = g.RS, PW = g.PW;
     const int NOT = 32 * (g.NWO + g.NWT);
+    const int NXW = 32 * (1 + g.NWT);
     const int W0T = 32 * (g.NWO + g.NWT);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rank = CLUSTER ? (int)cluster_rank() : 0;
@@ -793,6 +796,7 @@ __global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
                     timed_out = true;
                     set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
                 }
+                if constexpr (CLUSTER) cta_arrive(5, NXW);   // bp[s] of every label has arrived
                 const double n = warp_total(sm.gath + par * C, C, lane);
                 if (lane == 0) {
                     const int kk = sm.kbuf[u & 3];
@@ -833,14 +837,8 @@ __global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
             }
         } else if (ro.is_tr) {
             // ------------------------------------------- transposed transition
-            if constexpr (CLUSTER) {
-                if (!wait_values<CLUSTER>(sm, par, u, timed_out)) {
-                    timed_out = true;
-                    set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
-                }
-            } else {
-                cta_barrier(1, NOT);
-            }
+            if constexpr (CLUSTER) cta_barrier(5, NXW);
+            else cta_barrier(1, NOT);
             double v[CPL];
 #pragma unroll
             for (int m = 0; m < CPL; ++m) {
