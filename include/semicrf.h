@@ -21,9 +21,12 @@
  *   dX         float32 [B, T, C]    g_b * dlogZ_b/dx (through S and nu); 0 for t >= L_b
  *   dA         float64 [C, C]       sum_b g_b dlogZ_b/dA
  *   dD         float64 [K, C]       sum_b g_b dlogZ_b/dD
- *   score      float64 [B]          Viterbi score
- *   labels     int32   [B, T]       Viterbi label per position, -1 for t >= L_b
- *   seg_start  uint8   [B, T]       1 where a Viterbi segment begins, else 0
+ *   score      float64 [B]          Viterbi score (or a gold segmentation's score)
+ *   labels     int32   [B, T]       label per position (Viterbi output, or a gold
+ *                                   segmentation's input); -1 for t >= L_b in outputs
+ *   seg_start  uint8   [B, T]       1 where a segment begins, else 0
+ *   mu         float32 [B, T, C]    posterior coverage P(position lies in a segment of label c)
+ *   pstart     float32 [B, T]       posterior probability that a segment begins at t
  *
  * Ownership and execution: every data pointer is caller-owned DEVICE memory
  * (except where a function says otherwise).  The library allocates nothing and
@@ -60,7 +63,8 @@ typedef enum {
     SEMICRF_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed        */
     SEMICRF_ERR_DEVICE_TIMEOUT = 5,     /* a bounded device-side wait expired          */
     SEMICRF_ERR_DEVICE_RANGE = 6,       /* device saw a non-finite normaliser          */
-    SEMICRF_ERR_INVALID_LENGTH = 7      /* device saw a length outside [1, T]          */
+    SEMICRF_ERR_INVALID_LENGTH = 7,     /* device saw a length outside [1, T]          */
+    SEMICRF_ERR_INVALID_SEGMENTATION = 8 /* device saw a malformed gold segmentation   */
 } semicrf_status;
 
 /* Problem dimensions.  ckpt_interval is the checkpoint spacing Delta in positions
@@ -149,6 +153,53 @@ semicrf_status semicrf_viterbi(const semicrf_dims *dims, const double *S, const 
                                const float *D, const int32_t *lengths, double *score,
                                int32_t *labels, uint8_t *seg_start, void *ws,
                                size_t ws_bytes, void *stream);
+
+/*
+ * Posterior marginals (abstract: uncertainty estimates at segment boundaries;
+ * technical summary 2.C: the marginals the backward pass forms):
+ *   mu[b,u,c]   = P(position u lies in a segment labelled c)    (u < L_b; 0 beyond)
+ *   pstart[b,t] = P(a segment begins at t) = sum_c P(a segment of label c begins at t)
+ *                 (t < L_b; 0 beyond; pstart[b,0] = 1)
+ * Either output may be NULL.  Runs the recompute and backward passes of
+ * semicrf_backward on the forward's workspace (pass ws unchanged from the
+ * matching semicrf_forward) and forms no parameter gradients.
+ */
+semicrf_status semicrf_posteriors(const semicrf_dims *dims, const double *S, const float *A,
+                                  const float *D, const int32_t *lengths, void *ws,
+                                  size_t ws_bytes, float *mu, float *pstart, void *stream);
+
+/*
+ * Score of given ("gold") segmentations, the term the training loss subtracts
+ * from log Z (technical summary section 3: negative log-likelihood
+ * log Z - score(y*)).  Segment i of sequence b starts at a position s with
+ * seg_start[b,s] = 1 (seg_start[b,0] must be 1), ends at the next start or at
+ * L_b, has length at most K and label c = labels[b,s], which every position of
+ * the segment must carry (0 <= c < C).  Then
+ *   score[b] = sum_i (S[b,e_i,c_i] - S[b,s_i,c_i] + D[e_i-s_i-1,c_i]) + sum_{i>=2} A[c_{i-1},c_i].
+ * A malformed segmentation records SEMICRF_ERR_INVALID_SEGMENTATION in the
+ * workspace status (its score is then unspecified).  ws: a SEMICRF_WS_TRAIN
+ * workspace (its status word and count buffers are used).
+ */
+semicrf_status semicrf_gold_score(const semicrf_dims *dims, const double *S, const float *A,
+                                  const float *D, const int32_t *lengths, const int32_t *labels,
+                                  const uint8_t *seg_start, double *score, void *ws,
+                                  size_t ws_bytes, void *stream);
+
+/*
+ * Gradient of sum_b g_b score[b] (g = grad_score, NULL: ones) for the same
+ * segmentations, ADDED to dX, dA, dD (so that after semicrf_backward with
+ * weights g and this call with weights -g they hold the gradient of the
+ * negative log-likelihood):
+ *   dX[b,u,c] += g_b (1[u lies in a segment labelled c] - n_{b,c} / L_b)   (u < L_b)
+ *   dA[c',c]  += sum_b g_b * (number of c' -> c transitions in b)
+ *   dD[d-1,c] += sum_b g_b * (number of segments of length d and label c in b)
+ * where n_{b,c} counts the positions labelled c (the path through nu).  Checks
+ * the segmentations as semicrf_gold_score does.
+ */
+semicrf_status semicrf_gold_backward(const semicrf_dims *dims, const int32_t *lengths,
+                                     const int32_t *labels, const uint8_t *seg_start,
+                                     const double *grad_score, float *dX, double *dA, double *dD,
+                                     void *ws, size_t ws_bytes, void *stream);
 
 /* Zero the device status word in ws (asynchronous on stream). */
 semicrf_status semicrf_clear_device_status(void *ws, void *stream);

@@ -44,7 +44,7 @@ def _load():
         P = ctypes.c_void_p
         i = ctypes.c_int
         lib.oracle_prefix.argtypes = [i, i, i, P, P, i, P, P]
-        lib.oracle_factorised.argtypes = [i, i, i, i, P, P, P, P, i, i, P, P, P, P, P, P, P, i]
+        lib.oracle_factorised.argtypes = [i, i, i, i, P, P, P, P, i, i, P, P, P, P, P, P, P, P, i]
         lib.oracle_logz.argtypes = [i, i, i, i, P, P, P, P, i, P, i]
         lib.oracle_edge_direct.argtypes = [i, i, i, i, P, P, P, P, i, i, P, P, P, P, P, P, i]
         lib.oracle_viterbi.argtypes = [i, i, i, i, P, P, P, P, i, P, P, P, i]
@@ -87,8 +87,9 @@ def prefix(x, lengths, centre=True):
 
 
 def factorised(x, A, D, lengths, centre=True, detach_nu=False, grad_logZ=None,
-               want_mu=False, nthreads=0):
-    """log Z, backward log Z, dX, dA, dD (and coverage mu) from the factorised tier."""
+               want_mu=False, want_pstart=False, nthreads=0):
+    """log Z, backward log Z, dX, dA, dD (and coverage mu, start probability
+    pstart) from the factorised tier."""
     x, A, D, lengths, B, T, K, C = _prep(x, A, D, lengths)
     g = None if grad_logZ is None else np.ascontiguousarray(grad_logZ, dtype=np.float64)
     logZ = np.empty(B, np.float64)
@@ -97,12 +98,15 @@ def factorised(x, A, D, lengths, centre=True, detach_nu=False, grad_logZ=None,
     dA = np.empty((C, C), np.float64)
     dD = np.empty((K, C), np.float64)
     mu = np.empty((B, T, C), np.float64) if want_mu else None
+    ps = np.empty((B, T), np.float64) if want_pstart else None
     _check(_load().oracle_factorised(B, T, K, C, _p(x), _p(A), _p(D), _p(lengths), int(centre),
                                      int(detach_nu), _p(g), _p(logZ), _p(logZ_bwd), _p(dX),
-                                     _p(dA), _p(dD), _p(mu), int(nthreads)))
+                                     _p(dA), _p(dD), _p(mu), _p(ps), int(nthreads)))
     out = dict(logZ=logZ, logZ_bwd=logZ_bwd, dX=dX, dA=dA, dD=dD)
     if want_mu:
         out["mu"] = mu
+    if want_pstart:
+        out["pstart"] = ps
     return out
 
 
@@ -143,6 +147,34 @@ def viterbi(x, A, D, lengths, centre=True, nthreads=0):
     _check(_load().oracle_viterbi(B, T, K, C, _p(x), _p(A), _p(D), _p(lengths), int(centre),
                                   _p(score), _p(labels), _p(seg_start), int(nthreads)))
     return score, labels, seg_start
+
+
+def path_grads(x, A, D, lengths, labels, seg_start, centre=True, grad=None):
+    """Gradient of sum_b g_b path_score_b with respect to x, A, D, from the
+    definition: the score is linear in x (through the segment sums and nu), in A
+    (one term per transition) and in D (one term per segment)."""
+    x = np.asarray(x, np.float64)
+    B, T, C = x.shape
+    K = np.asarray(D).shape[0]
+    dX = np.zeros((B, T, C))
+    dA = np.zeros((C, C))
+    dD = np.zeros((K, C))
+    for b in range(B):
+        g = 1.0 if grad is None else float(grad[b])
+        L = int(lengths[b])
+        starts = [s for s in range(L) if seg_start[b, s]]
+        ends = starts[1:] + [L]
+        prev = None
+        for s, e in zip(starts, ends):
+            c = int(labels[b, s])
+            dX[b, s:e, c] += g                    # d/dx of sum_{u=s}^{e-1} x[u,c]
+            if centre:
+                dX[b, :L, c] -= g * (e - s) / L   # d/dx of -(e-s) nu[c], nu = mean over u < L
+            dD[e - s - 1, c] += g
+            if prev is not None:
+                dA[prev, c] += g
+            prev = c
+    return dX, dA, dD
 
 
 def path_score(x, A, D, lengths, labels, seg_start, centre=True):

@@ -50,7 +50,8 @@ def enumerate_sequence(x, A, D, L, centre=True):
     """Exact quantities for one sequence by enumeration.
 
     x: [T, C] (only the first L rows are used).  Returns dict with logZ, dA [C,C],
-    dD [K,C], mu [L,C] (coverage), dX [L,C] (gradient w.r.t. x, including the
+    dD [K,C], mu [L,C] (coverage), pstart [L] (probability that a segment
+    begins at each position), dX [L,C] (gradient w.r.t. x, including the
     path through the centring baseline when centre is set), best (score,
     list of (s, d, c)).
     """
@@ -78,9 +79,15 @@ def enumerate_sequence(x, A, D, L, centre=True):
     dA = np.zeros((C, C))
     dD = np.zeros((K, C))
     mu = np.zeros((L, C))
+    pstart = np.zeros(L)
     for durs in comps:
         n = len(durs)
         P = np.exp(_score_grid(xc, A, D, durs) - logZ)
+        total = P.sum()        # probability of this set of boundaries (all labellings)
+        s = 0
+        for d in durs:
+            pstart[s] += total
+            s += d
         s = 0
         for i, d in enumerate(durs):
             axes = tuple(j for j in range(n) if j != i)
@@ -99,7 +106,8 @@ def enumerate_sequence(x, A, D, L, centre=True):
     for d, c in zip(durs, labs):
         segs.append((s, d, int(c)))
         s += d
-    return dict(logZ=float(logZ), dA=dA, dD=dD, mu=mu, dX=dX, best_score=best[0], best_segs=segs)
+    return dict(logZ=float(logZ), dA=dA, dD=dD, mu=mu, pstart=pstart, dX=dX, best_score=best[0],
+                best_segs=segs)
 
 
 def enumerate_batch(x, A, D, lengths, centre=True):
@@ -110,6 +118,7 @@ def enumerate_batch(x, A, D, lengths, centre=True):
     logZ = np.empty(B)
     dX = np.zeros((B, T, C))
     mu = np.zeros((B, T, C))
+    pstart = np.zeros((B, T))
     dA = np.zeros((C, C))
     dD = np.zeros((K, C))
     scores = np.empty(B)
@@ -121,13 +130,14 @@ def enumerate_batch(x, A, D, lengths, centre=True):
         logZ[b] = r["logZ"]
         dX[b, :L] = r["dX"]
         mu[b, :L] = r["mu"]
+        pstart[b, :L] = r["pstart"]
         dA += r["dA"]
         dD += r["dD"]
         scores[b] = r["best_score"]
         for s, d, c in r["best_segs"]:
             labels[b, s:s + d] = c
             seg_start[b, s] = 1
-    return dict(logZ=logZ, dX=dX, mu=mu, dA=dA, dD=dD, score=scores, labels=labels,
+    return dict(logZ=logZ, dX=dX, mu=mu, pstart=pstart, dA=dA, dD=dD, score=scores, labels=labels,
                 seg_start=seg_start)
 
 

@@ -116,11 +116,14 @@ int oracle_prefix(int B, int T, int C, const double *x, const int32_t *lengths,
  *           = sum_{s<=u} sum_d Pseg(s,d,c) - sum_{s+d<=u} Pseg(s,d,c)
  *   dlogZ/dx[u,c] = mu[u,c] - (1/L) sum_{u'<L} mu[u',c]   (the second term is the
  *                   path through nu; dropped when nu is detached or not used)
+ *   pstart[s] = P(a segment begins at s) = sum_c sum_d Pseg(s,d,c)   (abstract:
+ *               uncertainty estimates at segment boundaries)
  * ------------------------------------------------------------------------- */
 static void seq_factorised(int L, int T, int K, int C, const double *S,
                            const double *Ad, const double *Dd, int par,
                            double *logZ_out, double *logZ_bwd_out,
-                           double *mu /* [T*C] */, double *dA_b, double *dD_b)
+                           double *mu /* [T*C] */, double *pstart /* [T] or NULL */,
+                           double *dA_b, double *dD_b)
 {
     size_t n = (size_t)(L + 1) * C;
     double *al = calloc(n, sizeof(double));
@@ -209,6 +212,14 @@ static void seq_factorised(int L, int T, int K, int C, const double *S,
         }
         for (int u = L; u < T; ++u) mu[IDX2(u, c, C)] = 0.0;
     }
+    if (pstart) {
+        for (int s = 0; s < T; ++s) {
+            double p = 0.0;
+            if (s < L)
+                for (int c = 0; c < C; ++c) p += st[IDX2(s, c, C)];
+            pstart[s] = p;
+        }
+    }
     *logZ_out = logZ;
     *logZ_bwd_out = logZ_bwd;
     free(al); free(at); free(be); free(ga); free(st); free(en);
@@ -231,14 +242,14 @@ static void finish_dx(int L, int T, int C, int use_nu_path, double g, const doub
 
 /*
  * Factorised oracle over a batch.  Outputs: logZ[B], logZ_bwd[B], dX[B,T,C],
- * dA[C,C], dD[K,C] (all float64), optional mu[B,T,C].  grad_logZ may be NULL
+ * dA[C,C], dD[K,C] (all float64), optional mu[B,T,C] and pstart[B,T].  grad_logZ may be NULL
  * (weights 1).  centre: subtract nu; detach_nu: drop the gradient path through nu.
  * Returns 0, or 1 on an invalid length.
  */
 int oracle_factorised(int B, int T, int K, int C, const double *x, const double *A,
                       const double *D, const int32_t *lengths, int centre, int detach_nu,
                       const double *grad_logZ, double *logZ, double *logZ_bwd, double *dX,
-                      double *dA, double *dD, double *mu_out, int nthreads)
+                      double *dA, double *dD, double *mu_out, double *pstart_out, int nthreads)
 {
     for (int b = 0; b < B; ++b)
         if (lengths[b] < 1 || lengths[b] > T) return 1;
@@ -259,8 +270,8 @@ int oracle_factorised(int B, int T, int K, int C, const double *x, const double 
         double *mu = malloc(sizeof(double) * (size_t)T * C);
         double g = grad_logZ ? grad_logZ[b] : 1.0;
         seq_factorised(lengths[b], T, K, C, S + (size_t)b * (T + 1) * C, Ad, Dd, !outer,
-                       &logZ[b], &logZ_bwd[b], mu, dA_all + (size_t)b * C * C,
-                       dD_all + (size_t)b * K * C);
+                       &logZ[b], &logZ_bwd[b], mu, pstart_out ? pstart_out + (size_t)b * T : NULL,
+                       dA_all + (size_t)b * C * C, dD_all + (size_t)b * K * C);
         finish_dx(lengths[b], T, C, centre && !detach_nu, g, mu, dX + (size_t)b * T * C);
         if (mu_out) memcpy(mu_out + (size_t)b * T * C, mu, sizeof(double) * (size_t)T * C);
         free(mu);

@@ -19,6 +19,7 @@ from ._lib import (MAX_C, MAX_K, WS_SCAN, WS_TRAIN, WS_VITERBI, SemiCRFError, di
                    status_string)
 
 __all__ = ["workspace_bytes", "new_workspace", "prefix_scan", "prefix_scan_noalloc", "forward", "backward", "viterbi",
+           "posteriors", "gold_score", "gold_backward", "semicrf_nll",
            "logz_and_grads", "device_status", "clear_device_status", "last_launch_count",
            "SemiCRFError", "status_string", "MAX_C", "MAX_K", "WS_TRAIN", "WS_VITERBI", "WS_SCAN",
            "load_library"]
@@ -158,6 +159,58 @@ def viterbi(S, A, D, lengths, ws=None):
                                            _ptr(score), _ptr(labels), _ptr(seg), _ptr(ws), ws.numel(),
                                            _stream(S.device)), "viterbi")
     return score, labels, seg
+
+
+def posteriors(S, A, D, lengths, ws, ckpt_interval=0, want_mu=True, want_pstart=True):
+    """(mu [B,T,C] float32 or None, pstart [B,T] float32 or None): posterior coverage
+    of each label and probability that a segment begins at each position.  ws is
+    the workspace of the matching forward()."""
+    torch = _torch()
+    B, T1, C = S.shape
+    T = T1 - 1
+    K = D.shape[0]
+    mu = torch.empty((B, T, C), dtype=torch.float32, device=S.device) if want_mu else None
+    ps = torch.empty((B, T), dtype=torch.float32, device=S.device) if want_pstart else None
+    d = dims(B, T, K, C, ckpt_interval)
+    _lib.check(_lib.load().semicrf_posteriors(ctypes.byref(d), _ptr(S), _ptr(A), _ptr(D), _ptr(lengths),
+                                              _ptr(ws), ws.numel(), _ptr(mu), _ptr(ps), _stream(S.device)),
+               "posteriors")
+    return mu, ps
+
+
+def gold_score(S, A, D, lengths, labels, seg_start, ws):
+    """Score [B] float64 of the segmentations given by labels [B,T] int32 and
+    seg_start [B,T] uint8 (the Viterbi output format)."""
+    torch = _torch()
+    B, T1, C = S.shape
+    T = T1 - 1
+    K = D.shape[0]
+    _need(labels, torch.int32, (B, T), "labels")
+    _need(seg_start, torch.uint8, (B, T), "seg_start")
+    score = torch.empty(B, dtype=torch.float64, device=S.device)
+    d = dims(B, T, K, C)
+    _lib.check(_lib.load().semicrf_gold_score(ctypes.byref(d), _ptr(S), _ptr(A), _ptr(D), _ptr(lengths),
+                                              _ptr(labels), _ptr(seg_start), _ptr(score), _ptr(ws), ws.numel(),
+                                              _stream(S.device)), "gold_score")
+    return score
+
+
+def gold_backward(lengths, labels, seg_start, ws, dX, dA, dD, grad_score=None):
+    """Add the gradient of sum_b g_b score_b of the given segmentations to dX, dA, dD."""
+    B, T, C = dX.shape
+    K = dD.shape[0]
+    d = dims(B, T, K, C)
+    _lib.check(_lib.load().semicrf_gold_backward(ctypes.byref(d), _ptr(lengths), _ptr(labels), _ptr(seg_start),
+                                                 _ptr(grad_score), _ptr(dX), _ptr(dA), _ptr(dD), _ptr(ws),
+                                                 ws.numel(), _stream(dX.device)), "gold_backward")
+    return dX, dA, dD
+
+
+def semicrf_nll(x, A, D, lengths, labels, seg_start, ckpt_interval=0):
+    """Negative log-likelihood log Z_b - score_b(gold) [B] float64, differentiable
+    with respect to x, A and D (torch.autograd)."""
+    from .nll import SemiCRFNLL
+    return SemiCRFNLL.apply(x, A, D, lengths, labels, seg_start, ckpt_interval)
 
 
 def logz_and_grads(x, A, D, lengths, grad_logZ=None, ckpt_interval=0, ws=None):

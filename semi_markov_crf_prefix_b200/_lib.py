@@ -18,6 +18,7 @@ SEMICRF_ERR_CUDA = 4
 SEMICRF_ERR_DEVICE_TIMEOUT = 5
 SEMICRF_ERR_DEVICE_RANGE = 6
 SEMICRF_ERR_INVALID_LENGTH = 7
+SEMICRF_ERR_INVALID_SEGMENTATION = 8
 
 WS_TRAIN = 0
 WS_VITERBI = 1
@@ -52,6 +53,9 @@ SIGNATURES = {
     "semicrf_forward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _S, _P]),
     "semicrf_backward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P]),
     "semicrf_viterbi": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "semicrf_posteriors": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _S, _P, _P, _P]),
+    "semicrf_gold_score": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "semicrf_gold_backward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
     "semicrf_clear_device_status": (ctypes.c_int, [_P, _P]),
     "semicrf_get_device_status": (ctypes.c_int, [_P, _P]),
     "semicrf_status_string": (ctypes.c_char_p, [ctypes.c_int]),

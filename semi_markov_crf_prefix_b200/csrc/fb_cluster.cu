@@ -813,7 +813,8 @@ __global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
                 // mu_acc holds the coverage of x[s] by label c; moving to x[s-1] adds the
                 // segments ending at s and removes those starting at s
                 const size_t row = (rowbase + s) * C + c;
-                a.dX[((size_t)b * a.T + s) * C + c] = (float)mu_acc;
+                if (a.dX) a.dX[((size_t)b * a.T + s) * C + c] = (float)mu_acc;
+                if (a.stst) a.stst[row] = start;
                 musum += mu_acc;
                 if (s >= 1) {
                     const double q = sm.qbuf[lc];

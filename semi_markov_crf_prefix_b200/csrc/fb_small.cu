@@ -472,7 +472,8 @@ __global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
                 n = 0.0;
                 for (int cc = 0; cc < C; ++cc) n += sm.xsh[par * 32 + cc];
             }
-            if (act) a.dX[((size_t)b * a.T + s) * C + c] = (float)mu_acc;
+            if (act && a.dX) a.dX[((size_t)b * a.T + s) * C + c] = (float)mu_acc;
+            if (act && a.stst) a.stst[(rowbase + s) * C + c] = start;
             musum += mu_acc;
             if (s == 0) {
                 if (lane == 0) a.logzb[b] = kLn2 * (double)kb + log(n);

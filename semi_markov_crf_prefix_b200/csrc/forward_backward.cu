@@ -96,6 +96,32 @@ __global__ void finalise_dx(FbArgs a)
     }
 }
 
+// Posterior outputs: zero mu beyond L_b; pstart[b,t] = sum_c P(start at t, label c).
+__global__ void posterior_finalise(FbArgs a, float *mu, float *pstart)
+{
+    const size_t nmu = mu ? (size_t)a.B * a.T * a.C : 0;
+    const size_t nps = pstart ? (size_t)a.B * a.T : 0;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < nmu + nps;
+         i += (size_t)gridDim.x * blockDim.x) {
+        if (i < nmu) {
+            const size_t bt = i / a.C;
+            const int u = (int)(bt % a.T), b = (int)(bt / a.T);
+            const int L = a.lengths[b];
+            if (L < 1 || L > a.T || u >= L) mu[i] = 0.0f;
+        } else {
+            const size_t bt = i - nmu;
+            const int t = (int)(bt % a.T), b = (int)(bt / a.T);
+            const int L = a.lengths[b];
+            double p = 0.0;
+            if (L >= 1 && L <= a.T && t < L) {
+                const double *row = a.stst + ((size_t)b * (a.T + 1) + t) * a.C;
+                for (int c = 0; c < a.C; ++c) p += row[c];
+            }
+            pstart[bt] = (float)p;
+        }
+    }
+}
+
 }  // namespace
 
 // Which kernel family runs: the warp-per-sequence kernels when the shape allows,
@@ -146,6 +172,26 @@ cudaError_t launch_backward(const Plan &p, const FbArgs &a, cudaStream_t st, int
     finalise_dx<<<blocks, 256, 0, st>>>(a);
     prof_after(st);
     *launches += small ? 4 : 6;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_posteriors(const FbArgs &a0, float *mu, float *pstart, cudaStream_t st, int *launches)
+{
+    FbArgs a = a0;
+    a.dX = mu;   // raw coverage; the parameter gradients are not formed
+    const bool small = use_small(a.K, a.C);
+    cudaError_t e = small ? launch_small(a, st, 1) : launch_cl_forward(a, st, true);
+    if (e != cudaSuccess) return e;
+    e = small ? launch_small(a, st, 2) : launch_cl_backward(a, st);
+    if (e != cudaSuccess) return e;
+    const size_t n = (mu ? (size_t)a.B * a.T * a.C : 0) + (pstart ? (size_t)a.B * a.T : 0);
+    int blocks = (int)((n + 255) / 256);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    prof_before(st);
+    posterior_finalise<<<blocks, 256, 0, st>>>(a, mu, pstart);
+    prof_after(st);
+    *launches += 3;
     return cudaGetLastError();
 }
 

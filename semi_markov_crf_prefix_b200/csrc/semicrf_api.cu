@@ -125,6 +125,10 @@ bool make_layout(const semicrf_dims &d, int what, const Plan &p, Layout *out)
         cl_grad_splits(d.B, d.T, d.K, d.C, &L.nsD, &L.nsA);
         L.partD = take((size_t)L.nsD * K * C * 8);
         L.partA = take((size_t)L.nsA * C * C * 8);
+        L.stst = take(B * (T + 1) * C * 8);
+        L.gcA = take(B * C * C * 4);
+        L.gcD = take(B * K * C * 4);
+        L.gcN = take(B * C * 4);
         L.musum = take(B * C * 8);
         L.mures = take(B * C * 8);
         L.logzb = take(B * 8);
@@ -309,6 +313,85 @@ semicrf_status semicrf_backward(const semicrf_dims *dims, const double *S, const
     return finish(e, n);
 }
 
+semicrf_status semicrf_posteriors(const semicrf_dims *dims, const double *S, const float *A, const float *D,
+                                  const int32_t *lengths, void *ws, size_t ws_bytes, float *mu, float *pstart,
+                                  void *stream)
+{
+    Plan p;
+    Layout lay;
+    semicrf_status s = prepare(dims, SEMICRF_WS_TRAIN, ws, ws_bytes, &p, &lay);
+    if (s != SEMICRF_OK) return s;
+    if (!S || !A || !D || !lengths) return SEMICRF_ERR_INVALID_ARG;
+    FbArgs a = fb_args(dims, lay, ws);
+    a.S = S;
+    a.A = A;
+    a.D = D;
+    a.lengths = lengths;
+    a.stst = at<double>(ws, lay.stst);
+    int n = 0;
+    cudaError_t e = launch_posteriors(a, mu, pstart, static_cast<cudaStream_t>(stream), &n);
+    return finish(e, n);
+}
+
+namespace {
+GoldArgs gold_args(const semicrf_dims *dims, const Layout &lay, void *ws, const int32_t *lengths,
+                   const int32_t *labels, const uint8_t *seg_start)
+{
+    GoldArgs g;
+    memset(&g, 0, sizeof(g));
+    g.B = dims->B;
+    g.T = dims->T;
+    g.K = dims->K;
+    g.C = dims->C;
+    g.lengths = lengths;
+    g.labels = labels;
+    g.seg_start = seg_start;
+    g.cntA = at<int32_t>(ws, lay.gcA);
+    g.cntD = at<int32_t>(ws, lay.gcD);
+    g.cntN = at<int32_t>(ws, lay.gcN);
+    g.status = at<int32_t>(ws, lay.status);
+    return g;
+}
+}  // namespace
+
+semicrf_status semicrf_gold_score(const semicrf_dims *dims, const double *S, const float *A, const float *D,
+                                  const int32_t *lengths, const int32_t *labels, const uint8_t *seg_start,
+                                  double *score, void *ws, size_t ws_bytes, void *stream)
+{
+    Plan p;
+    Layout lay;
+    semicrf_status s = prepare(dims, SEMICRF_WS_TRAIN, ws, ws_bytes, &p, &lay);
+    if (s != SEMICRF_OK) return s;
+    if (!S || !A || !D || !lengths || !labels || !seg_start || !score) return SEMICRF_ERR_INVALID_ARG;
+    GoldArgs g = gold_args(dims, lay, ws, lengths, labels, seg_start);
+    g.S = S;
+    g.A = A;
+    g.D = D;
+    g.score = score;
+    int n = 0;
+    cudaError_t e = launch_gold_score(g, static_cast<cudaStream_t>(stream), &n);
+    return finish(e, n);
+}
+
+semicrf_status semicrf_gold_backward(const semicrf_dims *dims, const int32_t *lengths, const int32_t *labels,
+                                     const uint8_t *seg_start, const double *grad_score, float *dX, double *dA,
+                                     double *dD, void *ws, size_t ws_bytes, void *stream)
+{
+    Plan p;
+    Layout lay;
+    semicrf_status s = prepare(dims, SEMICRF_WS_TRAIN, ws, ws_bytes, &p, &lay);
+    if (s != SEMICRF_OK) return s;
+    if (!lengths || !labels || !seg_start || !dX || !dA || !dD) return SEMICRF_ERR_INVALID_ARG;
+    GoldArgs g = gold_args(dims, lay, ws, lengths, labels, seg_start);
+    g.grad = grad_score;
+    g.dX = dX;
+    g.dA = dA;
+    g.dD = dD;
+    int n = 0;
+    cudaError_t e = launch_gold_backward(g, static_cast<cudaStream_t>(stream), &n);
+    return finish(e, n);
+}
+
 semicrf_status semicrf_viterbi(const semicrf_dims *dims, const double *S, const float *A, const float *D,
                                const int32_t *lengths, double *score, int32_t *labels,
                                uint8_t *seg_start, void *ws, size_t ws_bytes, void *stream)
@@ -366,6 +449,7 @@ const char *semicrf_status_string(semicrf_status s)
     case SEMICRF_ERR_DEVICE_TIMEOUT: return "device wait timed out";
     case SEMICRF_ERR_DEVICE_RANGE: return "non-finite value on device";
     case SEMICRF_ERR_INVALID_LENGTH: return "sequence length outside [1, T]";
+    case SEMICRF_ERR_INVALID_SEGMENTATION: return "malformed gold segmentation";
     }
     return "unknown status";
 }

@@ -69,6 +69,10 @@ struct Layout {
     int nsD = 0, nsA = 0;   // partial-sum splits of the dD and dA contractions
     size_t partD = 0;       // double [nsD][K][C]
     size_t partA = 0;       // double [nsA][C][C]
+    size_t stst = 0;        // double [B][T+1][C]  P(segment of label c starts at s) (posteriors)
+    size_t gcA = 0;         // int32  [B][C][C]    gold transition counts
+    size_t gcD = 0;         // int32  [B][K][C]    gold duration counts
+    size_t gcN = 0;         // int32  [B][C]       gold positions per label
     size_t musum = 0;       // double [B][C]
     size_t mures = 0;       // double [B][C]
     size_t logzb = 0;       // double [B]
@@ -117,6 +121,7 @@ struct FbArgs {
     double *Vst, *bpst, *partD, *partA;
     int32_t *rbst, *kbst;
     int nsD, nsA;
+    double *stst;   // when set, the backward stores the start marginals (posteriors)
     float *dX;
     double *dA, *dD;
     int32_t *status;
@@ -164,5 +169,26 @@ struct VitArgs {
     int32_t *status;
 };
 cudaError_t launch_viterbi(const Plan &p, const VitArgs &a, cudaStream_t st, int *launches);
+
+// Posterior marginals: the recompute and backward chains with a.dX = mu (raw
+// coverage, or NULL) and a.stst set, then one kernel for pstart and the padding.
+cudaError_t launch_posteriors(const FbArgs &a, float *mu, float *pstart, cudaStream_t st, int *launches);
+
+// Gold segmentations (gold.cu).
+struct GoldArgs {
+    int B, T, K, C;
+    const double *S;
+    const float *A, *D;
+    const int32_t *lengths, *labels;
+    const uint8_t *seg_start;
+    const double *grad;   // backward weights, NULL: ones
+    double *score;
+    float *dX;
+    double *dA, *dD;
+    int32_t *cntA, *cntD, *cntN;
+    int32_t *status;
+};
+cudaError_t launch_gold_score(const GoldArgs &a, cudaStream_t st, int *launches);
+cudaError_t launch_gold_backward(const GoldArgs &a, cudaStream_t st, int *launches);
 
 }  // namespace semicrf

@@ -25,6 +25,9 @@ Readings of the distribution recipe (standard deviations throughout):
   * large: a per-label mean offset 2 * (c + 1) ** -1.1 (Zipf exponent 1.1,
     amplitude 2 so that label 0 matches the +2 "outside" offset of the
     named-entity workload).
+  * stress: the scale test of one million positions with K = 200 (the pages'
+    scalability claim); C = 24 and the genomic recipe (geometric segments of
+    mean 200 with +1.5 on the true label) are this module's choice.
 """
 from __future__ import annotations
 
@@ -67,6 +70,7 @@ CONFIGS = {
     "speech": (16, 4000, 64, 128),
     "genomic": (1, 100_000, 1000, 24),
     "large": (4, 200_000, 512, 256),
+    "stress": (1, 1_000_000, 200, 24),
 }
 
 
@@ -132,7 +136,7 @@ def genomic_segments(rng, T, C, mean_len=200.0):
     return np.array(starts, dtype=np.int64), np.array(labels, dtype=np.int64)
 
 
-def _genomic(B, T, K, C, seed, mean_len=200.0):
+def _genomic(B, T, K, C, seed, mean_len=200.0, name="genomic"):
     rng = _rng(seed)
     x = _normal32(rng, (B, T, C))
     A = _normal32(rng, (C, C), 0.3)
@@ -143,7 +147,7 @@ def _genomic(B, T, K, C, seed, mean_len=200.0):
         for s, e, c in zip(starts, ends, labels):
             x[b, s:e, c] += np.float32(1.5)
     lengths = np.full(B, T, dtype=np.int32)
-    return Workload("genomic", B, T, K, C, x, A, D, lengths, seed)
+    return Workload(name, B, T, K, C, x, A, D, lengths, seed)
 
 
 def _large(B, T, K, C, seed):
@@ -178,6 +182,8 @@ def make_workload(name: str, seed: int = 0, *, B=None, T=None, K=None, C=None) -
         return _genomic(B, T, K, C, seed)
     if name == "large":
         return _large(B, T, K, C, seed)
+    if name == "stress":
+        return _genomic(B, T, K, C, seed, name="stress")
     raise KeyError(name)
 
 

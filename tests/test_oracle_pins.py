@@ -14,6 +14,9 @@ transposed transition) fails at least one of them:
       per-position constants)
   P8  reversal symmetry
   P9  Viterbi: enumeration, path score recomputed from the definition, score <= log Z
+  P10 segment-start probabilities: enumeration, all-zero closed form, expected
+      number of segments
+  P11 gold-path gradient: finite differences of the path score, feature counts
   M8  drift of the cumulative scores: centred << uncentred, S[L] = 0
 """
 import math
@@ -374,3 +377,98 @@ def test_m8_centring_controls_drift(ner):
     for b in range(w.B):
         L = int(w.lengths[b])
         np.testing.assert_allclose(nu[b], w.x[b, :L].astype(np.float64).mean(axis=0), rtol=1e-12)
+
+
+# -------------------------------------------------------------------------- P10
+def test_p10_start_probabilities_bruteforce(tiny10):
+    w = tiny10
+    e = bf.enumerate_batch(w.x, w.A, w.D, w.lengths)
+    f = oracle.factorised(w.x, w.A, w.D, w.lengths, want_pstart=True)
+    np.testing.assert_allclose(f["pstart"], e["pstart"], rtol=0, atol=1e-12)
+    # a ragged batch: zero beyond L_b, one at 0
+    w2 = wl.random_small(seed=31, B=3, T=9, K=4, C=3, ragged=True)
+    e2 = bf.enumerate_batch(w2.x, w2.A, w2.D, w2.lengths)
+    f2 = oracle.factorised(w2.x, w2.A, w2.D, w2.lengths, want_pstart=True)
+    np.testing.assert_allclose(f2["pstart"], e2["pstart"], rtol=0, atol=1e-12)
+    for b in range(w2.B):
+        assert f2["pstart"][b, 0] == pytest.approx(1.0, abs=1e-13)
+        assert np.all(f2["pstart"][b, w2.lengths[b]:] == 0.0)
+
+
+@pytest.mark.parametrize("L,K,C", [(7, 7, 3), (12, 20, 4)])
+def test_p10_start_probabilities_zero_scores(L, K, C):
+    # all-zero scores with K >= L: each interior boundary independently present
+    # with probability C / (1 + C)
+    f = oracle.factorised(np.zeros((1, L, C)), np.zeros((C, C)), np.zeros((K, C)),
+                          np.array([L], np.int32), want_pstart=True)
+    expect = np.full(L, C / (1 + C))
+    expect[0] = 1.0
+    np.testing.assert_allclose(f["pstart"][0], expect, rtol=1e-12)
+
+
+def test_p10_expected_segment_count(ner):
+    # each segment has exactly one start: sum_s P(start at s) = E[#segments] = sum dD
+    w = wl.make_workload("ner", B=4, T=128)
+    f = oracle.factorised(w.x, w.A, w.D, w.lengths, want_pstart=True)
+    for b in range(w.B):
+        fb = oracle.factorised(w.x[b:b + 1], w.A, w.D, w.lengths[b:b + 1])
+        np.testing.assert_allclose(f["pstart"][b].sum(), fb["dD"].sum(), rtol=1e-12)
+
+
+# -------------------------------------------------------------------------- P11
+def _random_segmentation(rng, L, K, C, T):
+    labels = np.full(T, -1, np.int32)
+    seg = np.zeros(T, np.uint8)
+    s = 0
+    while s < L:
+        d = int(rng.integers(1, min(K, L - s) + 1))
+        c = int(rng.integers(0, C))
+        labels[s:s + d] = c
+        seg[s] = 1
+        s += d
+    return labels, seg
+
+
+def test_p11_path_gradient_finite_differences(tiny):
+    w = tiny
+    rng = np.random.default_rng(5)
+    labels = np.zeros((w.B, w.T), np.int32)
+    seg = np.zeros((w.B, w.T), np.uint8)
+    for b in range(w.B):
+        labels[b], seg[b] = _random_segmentation(rng, int(w.lengths[b]), w.K, w.C, w.T)
+    g = np.array([0.7, -1.3])
+    dX, dA, dD = oracle.path_grads(w.x, w.A, w.D, w.lengths, labels, seg, grad=g)
+
+    def f(x, A, D):
+        return float(np.dot(g, oracle.path_score(x, A, D, w.lengths, labels, seg)))
+
+    x0, A0, D0 = (np.asarray(v, np.float64).copy() for v in (w.x, w.A, w.D))
+    h = 1e-3   # the score is linear: central differences are exact up to rounding
+    for (arr, grad) in ((x0, dX), (A0, dA), (D0, dD)):
+        num = np.zeros_like(arr)
+        it = np.nditer(arr, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            old = arr[i]
+            arr[i] = old + h
+            fp = f(x0, A0, D0)
+            arr[i] = old - h
+            fm = f(x0, A0, D0)
+            arr[i] = old
+            num[i] = (fp - fm) / (2 * h)
+        np.testing.assert_allclose(grad, num, rtol=0, atol=1e-9)
+
+
+def test_p11_path_counts(ner):
+    w = wl.make_workload("ner", B=3, T=100)
+    rng = np.random.default_rng(9)
+    labels = np.zeros((w.B, w.T), np.int32)
+    seg = np.zeros((w.B, w.T), np.uint8)
+    for b in range(w.B):
+        labels[b], seg[b] = _random_segmentation(rng, int(w.lengths[b]), w.K, w.C, w.T)
+    dX, dA, dD = oracle.path_grads(w.x, w.A, w.D, w.lengths, labels, seg)
+    nseg = int(seg.sum())
+    assert dD.sum() == pytest.approx(nseg)
+    assert dA.sum() == pytest.approx(nseg - w.B)
+    assert (np.arange(1, w.K + 1)[:, None] * dD).sum() == pytest.approx(int(w.lengths.sum()))
+    np.testing.assert_allclose(dX.sum(axis=1), 0.0, atol=1e-12)   # centring: zero sum over positions
