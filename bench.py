@@ -195,9 +195,9 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     sc.load_library()
 
-    w = wl.make_workload(args.config, seed=args.seed)
+    w = wl.make_workload(args.config, seed=args.seed, B=args.B, T=args.T)
     if rank > 0:   # data-parallel: every rank its own emissions and lengths, shared A and D
-        own = wl.make_workload(args.config, seed=args.seed + 1000 * rank)
+        own = wl.make_workload(args.config, seed=args.seed + 1000 * rank, B=args.B, T=args.T)
         w.x, w.lengths = own.x, own.lengths
     B, T, K, C = w.B, w.T, w.K, w.C
     sumL, terms_pass, bytes_path = algorithmic(w)
@@ -351,7 +351,7 @@ def run_gpu(args):
         achieved = work_flop[dom] / (per_launch_ms / 1e3) / 1e12
         roof = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": fp64_peak_tflops,
                 "unit": "TFLOP/s", "frac": achieved / fp64_peak_tflops,
-                "traffic": recorded_traffic(dom, args.config),
+                "traffic": recorded_traffic(dom, args.config) if args.B is None and args.T is None else None,
                 "peak_source": f"derived: {N_SM} SMs x {FP64_FMA_PER_SM_CLK} FP64 FMA/clk x 2 x {sm_max:.0f} MHz",
                 "work": "2 flop per (log-sum-exp, +) term: sum_b L_b (K*C + C*C) terms per launch"}
     else:
@@ -409,7 +409,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return None
-    w = wl.make_workload(args.config, seed=args.seed)
+    w = wl.make_workload(args.config, seed=args.seed, B=args.B, T=args.T)
     budget = max(0.5, args.cpu_budget / max(1, args.steps))
     for _ in range(args.warmup if args.warmup < 2 else 1):
         oracle_sample(w, budget_s=0.01)
@@ -444,6 +444,8 @@ def main():
     ap.add_argument("--config", default="ner", choices=[k for k in wl.CONFIGS if k != "tiny10"])
     ap.add_argument("--ckpt", type=int, default=0, help="checkpoint interval (0: ceil(sqrt(T)))")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--B", type=int, default=None, help="override the workload's batch (small profiling cases)")
+    ap.add_argument("--T", type=int, default=None, help="override the workload's length (same recipe)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

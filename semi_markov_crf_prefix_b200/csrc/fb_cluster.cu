@@ -960,12 +960,16 @@ int pow2_ceil(int v)
 
 // One candidate geometry: G CTAs, LPL transition lanes per label, LPW window
 // lanes per label.  Returns false when it does not fit 1024 threads or shared
-// memory.  *cost estimates the cycles of one position from the latencies of
-// this part (a dependent FP64 operation ~33 cycles, a shared load ~55, a shuffle
-// level with its add ~58, the cluster exchange ~230): the owner-transition
-// chain and the window warps run in parallel, the slower one sets the pace.
-// Register classes that spill (more than 512 threads, or 32 transition terms
-// per lane with more than 256) pay extra.
+// memory.  *cost estimates the cycles of one position, calibrated on this part:
+// the owner-transition chain is about 2.5x the sum of its dependent latencies
+// (FP64 operation ~33 cycles, shared load ~55, shuffle level ~58, exchange
+// ~230 + C*G/2, at most 830: it grows with the values sent and the CTAs they
+// go to) plus
+// ~12 cycles of issue per transition
+// term; a window chunk of eight rows costs ~1000 cycles in context; every
+// resident warp adds ~25 cycles of contention; register classes that spill pay
+// extra (more above 512 threads).  The chain and the window warps run in
+// parallel, the slower one sets the pace.
 static bool cl_try(int K, int C, bool bwd, int G, int LPL, int LPW, ClGeom *out, double *cost)
 {
     ClGeom g;
@@ -1000,10 +1004,13 @@ static bool cl_try(int K, int C, bool bwd, int G, int LPL, int LPW, ClGeom *out,
         return l;
     };
     const int R = (rows + LPW - 1) / LPW;
-    const double chain = 33 + (G > 1 ? 230 + 10 * G : 40) + 55 + 33 * (1 + lg2(cpl)) + 58 * lg2(LPL) + 150;
-    const double window = ((R + 7) / 8) * 190.0 + 58 * lg2(LPW < 32 ? LPW : 32) + 60;
-    double c = chain > window ? chain : window;
-    if (maxt > 512 || (cpl == 32 && maxt > 256)) c += 400;   // register classes that spill
+    const double chain =
+        2.5 * (33 + (G > 1 ? 230 + (C * G < 1200 ? 0.5 * C * G : 600.0) : 40) + 55 + 33 * (1 + lg2(cpl)) +
+               58 * lg2(LPL) + 150 + 12 * cpl);
+    const double window = 1000.0 * ((R + 7) / 8) + 60 * lg2(LPW < 32 ? LPW : 32);
+    double c = (chain > window ? chain : window) + 25.0 * (g.NT / 32);
+    if (maxt > 512) c += 2000;                     // register classes that spill
+    else if (cpl == 32 && maxt > 256) c += 600;
     *out = g;
     *cost = c;
     return true;
