@@ -41,13 +41,12 @@ FP64_FMA_PER_SM_CLK = 64
 MUFU_PER_SM_CLK = 16
 HBM_FALLBACK_GBS = 6650.0
 SM_MAX_MHZ_FALLBACK = 1965.0
-# every kernel one step launches, in launch order: prefix_scan 3, forward 2, and a
-# backward of 4 (warp-per-sequence kernels, C, K <= 32) or 6 (cluster kernels, whose
-# dD and dA are separate contraction kernels)
+# every kernel one step launches, in launch order: prefix_scan 3, then
+# forward_backward 11 (both chains side by side in one launch, then the passes
+# over the stored rows)
 SCAN_NAMES = ["scan_partials", "scan_offsets", "scan_apply"]
-FWD_NAMES = ["exp_tables", "fwd_kernel"]
-BWD_NAMES = {4: ["fwd_recompute", "bwd_kernel", "finalise_params", "finalise_dx"],
-             6: ["fwd_recompute", "bwd_kernel", "dur_grad", "trans_grad", "finalise_params", "finalise_dx"]}
+FB_NAMES = ["exp_tables", "chains", "rows_rescale", "cov_delta", "cov_offsets", "cov_scan", "cov_musum",
+            "dur_grad", "trans_grad", "finalise_params", "finalise_dx"]
 
 
 def measured_peaks():
@@ -216,13 +215,7 @@ def run_gpu(args):
     dD = torch.empty((K, C), dtype=torch.float64, device=dev)
     flush = torch.empty(256 * 2**20 // 4, dtype=torch.float32, device=dev)
 
-    # the backward's kernel list depends on the kernel family the shape uses
-    sc.clear_device_status(ws)
-    sc.prefix_scan(x, lens, ws=ws, S=S, nu=nu)
-    sc.forward(S, A, D, lens, ws=ws, ckpt_interval=args.ckpt, logZ=logZ)
-    sc.backward(S, A, D, lens, ws, ckpt_interval=args.ckpt, dX=dX, dA=dA, dD=dD)
-    n_bwd = sc.last_launch_count()
-    KERNEL_NAMES = SCAN_NAMES + FWD_NAMES + BWD_NAMES[n_bwd]
+    KERNEL_NAMES = SCAN_NAMES + FB_NAMES
     # per-kernel events (recorded by the library around each launch)
     n_ev = 2 * len(KERNEL_NAMES)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
@@ -236,11 +229,8 @@ def run_gpu(args):
             lib.semicrf_set_profile_events(handles, 6)
         sc.prefix_scan(x, lens, ws=ws, S=S, nu=nu)
         if profile:
-            lib.semicrf_set_profile_events(ctypes_offset(handles, 6), 4)
-        sc.forward(S, A, D, lens, ws=ws, ckpt_interval=args.ckpt, logZ=logZ)
-        if profile:
-            lib.semicrf_set_profile_events(ctypes_offset(handles, 10), 2 * n_bwd)
-        sc.backward(S, A, D, lens, ws, ckpt_interval=args.ckpt, dX=dX, dA=dA, dD=dD)
+            lib.semicrf_set_profile_events(ctypes_offset(handles, 6), 2 * len(FB_NAMES))
+        sc.forward_backward(S, A, D, lens, ws=ws, logZ=logZ, dX=dX, dA=dA, dD=dD)
         if profile:
             lib.semicrf_set_profile_events(None, 0)
         if world > 1:
@@ -345,15 +335,15 @@ def run_gpu(args):
     fp64_peak_tflops = N_SM * FP64_FMA_PER_SM_CLK * 2 * sm_max * 1e6 / 1e12
     dom = max(kern_ms, key=kern_ms.get)
     per_launch_ms = kern_ms[dom] / args.steps
-    work_flop = {"fwd_kernel": 2 * terms_pass, "bwd_kernel": 2 * terms_pass,
-                 "fwd_recompute": 2 * terms_pass}
+    work_flop = {"chains": 2 * 2 * terms_pass}   # the forward and the backward pass
     if dom in work_flop:
         achieved = work_flop[dom] / (per_launch_ms / 1e3) / 1e12
         roof = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": fp64_peak_tflops,
                 "unit": "TFLOP/s", "frac": achieved / fp64_peak_tflops,
                 "traffic": recorded_traffic(dom, args.config) if args.B is None and args.T is None else None,
                 "peak_source": f"derived: {N_SM} SMs x {FP64_FMA_PER_SM_CLK} FP64 FMA/clk x 2 x {sm_max:.0f} MHz",
-                "work": "2 flop per (log-sum-exp, +) term: sum_b L_b (K*C + C*C) terms per launch"}
+                "work": "2 flop per (log-sum-exp, +) term: sum_b L_b (K*C + C*C) terms per pass, "
+                        "forward and backward pass in the one launch"}
     else:
         hbm = float(peaks.get("hbm_gbs", HBM_FALLBACK_GBS))
         nbytes = 4 * B * T * C + 8 * B * (T + 1) * C
@@ -373,7 +363,7 @@ def run_gpu(args):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.config, "B": B, "T": T, "K": K, "C": C,
-                   "ckpt_interval": args.ckpt or int(math.ceil(math.sqrt(T))), "seed": args.seed,
+                   "path": "forward_backward (both chains side by side, no checkpoints)", "seed": args.seed,
                    "sum_lengths": sumL, "valid_updates_per_s": world * w.valid_updates * args.steps / (total_ms / 1e3),
                    "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"dp{world}"},
         "roofline": roof,

@@ -144,6 +144,22 @@ semicrf_status semicrf_backward(const semicrf_dims *dims, const double *S, const
                                 float *dX, double *dA, double *dD, void *stream);
 
 /*
+ * Forward and backward in one call: log Z and the gradients of semicrf_backward
+ * (weights grad_logZ, NULL: ones), without checkpoints.  The forward chain and
+ * the backward (beta) chain run side by side -- the backward chain needs only
+ * S, A, D and the lengths -- and each stores its per-position rows; the
+ * marginals, coverage and parameter gradients are then parallel passes over
+ * them (technical summary 2.C computes the same quantities by checkpointed
+ * recompute, which semicrf_forward / semicrf_backward keep for callers that
+ * split the two).  Same workspace kind and outputs as the pair; the result
+ * equals theirs up to rounding order.
+ */
+semicrf_status semicrf_forward_backward(const semicrf_dims *dims, const double *S, const float *A,
+                                       const float *D, const int32_t *lengths, const double *grad_logZ,
+                                       void *ws, size_t ws_bytes, double *logZ, float *dX, double *dA,
+                                       double *dD, void *stream);
+
+/*
  * Viterbi: the forward recursion in (max, +), float64.  Ties pick the smallest
  * duration, then the smallest previous label; the final label is the smallest
  * reaching the maximum.  (The pages do not describe decoding; this follows the

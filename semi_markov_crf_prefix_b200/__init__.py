@@ -18,7 +18,8 @@ from . import _lib
 from ._lib import (MAX_C, MAX_K, WS_SCAN, WS_TRAIN, WS_VITERBI, SemiCRFError, dims,
                    status_string)
 
-__all__ = ["workspace_bytes", "new_workspace", "prefix_scan", "prefix_scan_noalloc", "forward", "backward", "viterbi",
+__all__ = ["workspace_bytes", "new_workspace", "prefix_scan", "prefix_scan_noalloc", "forward", "backward",
+           "forward_backward", "viterbi",
            "posteriors", "gold_score", "gold_backward", "semicrf_nll",
            "logz_and_grads", "device_status", "clear_device_status", "last_launch_count",
            "SemiCRFError", "status_string", "MAX_C", "MAX_K", "WS_TRAIN", "WS_VITERBI", "WS_SCAN",
@@ -159,6 +160,32 @@ def viterbi(S, A, D, lengths, ws=None):
                                            _ptr(score), _ptr(labels), _ptr(seg), _ptr(ws), ws.numel(),
                                            _stream(S.device)), "viterbi")
     return score, labels, seg
+
+
+def forward_backward(S, A, D, lengths, ws=None, grad_logZ=None, logZ=None, dX=None, dA=None, dD=None):
+    """(logZ, dX, dA, dD, ws): forward and backward chains side by side, then the
+    gradient passes (no checkpoints)."""
+    torch = _torch()
+    B, T1, C = S.shape
+    T = T1 - 1
+    K = D.shape[0]
+    _need(S, torch.float64, (B, T + 1, C), "S")
+    _need(A, torch.float32, (C, C), "A")
+    _need(D, torch.float32, (K, C), "D")
+    _need(lengths, torch.int32, (B,), "lengths")
+    if grad_logZ is not None:
+        _need(grad_logZ, torch.float64, (B,), "grad_logZ")
+    if ws is None:
+        ws = new_workspace(B, T, K, C, WS_TRAIN, device=S.device)
+    logZ = torch.empty(B, dtype=torch.float64, device=S.device) if logZ is None else logZ
+    dX = torch.empty((B, T, C), dtype=torch.float32, device=S.device) if dX is None else dX
+    dA = torch.empty((C, C), dtype=torch.float64, device=S.device) if dA is None else dA
+    dD = torch.empty((K, C), dtype=torch.float64, device=S.device) if dD is None else dD
+    d = dims(B, T, K, C)
+    _lib.check(_lib.load().semicrf_forward_backward(ctypes.byref(d), _ptr(S), _ptr(A), _ptr(D), _ptr(lengths),
+                                                    _ptr(grad_logZ), _ptr(ws), ws.numel(), _ptr(logZ), _ptr(dX),
+                                                    _ptr(dA), _ptr(dD), _stream(S.device)), "forward_backward")
+    return logZ, dX, dA, dD, ws
 
 
 def posteriors(S, A, D, lengths, ws, ckpt_interval=0, want_mu=True, want_pstart=True):

@@ -53,6 +53,7 @@ SIGNATURES = {
     "semicrf_forward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _S, _P]),
     "semicrf_backward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P]),
     "semicrf_viterbi": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "semicrf_forward_backward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P, _P]),
     "semicrf_posteriors": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _S, _P, _P, _P]),
     "semicrf_gold_score": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
     "semicrf_gold_backward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),

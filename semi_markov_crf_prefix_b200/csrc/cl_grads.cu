@@ -175,25 +175,145 @@ __global__ void __launch_bounds__(256) trans_grad_kernel(FbArgs a)
     }
 }
 
-// dD = exp(D) * sum_z partD[z],  dA = exp(A) * sum_z partA[z]   (splits in order)
+// dD = exp(D) * sum_z partD[z],  dA = exp(A) * sum_z partA[z]: one warp per
+// output, lane l adds the splits z = l, l+32, ... in order, then a fixed xor tree
+// (the result does not depend on scheduling).
 __global__ void cl_finalise_params(FbArgs a)
 {
     const int nA = a.C * a.C, nD = a.K * a.C;
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nA + nD; i += gridDim.x * blockDim.x) {
+    const int lane = threadIdx.x & 31;
+    const int w0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, nw = (gridDim.x * blockDim.x) >> 5;
+    for (int i = w0; i < nA + nD; i += nw) {
+        double s = 0.0;
         if (i < nA) {
-            double s = 0.0;
-            for (int z = 0; z < a.nsA; ++z) s += a.partA[(size_t)z * nA + i];
-            a.dA[i] = exp((double)a.A[i]) * s;
+            for (int z = lane; z < a.nsA; z += 32) s += a.partA[(size_t)z * nA + i];
         } else {
-            const int k = i - nA;
-            double s = 0.0;
-            for (int z = 0; z < a.nsD; ++z) s += a.partD[(size_t)z * nD + k];
-            a.dD[k] = exp((double)a.D[k]) * s;
+            for (int z = lane; z < a.nsD; z += 32) s += a.partD[(size_t)z * nD + (i - nA)];
+        }
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) {
+            if (i < nA) a.dA[i] = exp((double)a.A[i]) * s;
+            else a.dD[i - nA] = exp((double)a.D[i - nA]) * s;
         }
     }
 }
 
 int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// Rows the forward stored unscaled (cU = U, eU = r, cA = a', eA = k) become the
+// recompute's convention once log Z = ln2 kZ + logn is known:
+//   cU *= exp(-logn), eU -= kZ, cA *= exp(-logn), eA -= kZ     (t in [1, L])
+__global__ void rows_rescale(FbArgs a)
+{
+    const size_t n = (size_t)a.B * (a.T + 1) * a.C;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const size_t bt = i / a.C;
+        const int t = (int)(bt % (a.T + 1)), b = (int)(bt / (a.T + 1));
+        const int L = a.lengths[b];
+        if (L < 1 || L > a.T || t < 1 || t > L) continue;
+        const int kZ = a.lz[b].k;
+        const double cz = exp(-a.lz[b].logn);
+        if (t < L) {
+            a.cU[i] *= cz;
+            a.eU[i] -= kZ;
+        }
+        a.cA[i] *= cz;
+        if ((int)(i % a.C) == 0) a.eA[bt] -= kZ;
+    }
+}
+
+// Segment start and end marginals of label c at position u from the stored rows:
+//   start(u) = exp(at[u] - S[u] - log Z) exp(be[u]) exp(S[u])   (a segment begins at u)
+//   end(u)   = exp(al[u] - log Z) exp(ga[u])                     (a segment ends at u, u >= 1)
+// with every factor a mantissa and a power of two, so the product is exact up to
+// rounding whatever the references.
+__device__ __forceinline__ double seg_start_marg(const FbArgs &a, size_t rowbase, int b, int u, int c)
+{
+    const size_t ix = (rowbase + u) * a.C + c;
+    const double bp = a.bpst[ix], es = a.tES[ix];
+    const int kb = a.kbst[rowbase + u], m = a.tM[ix];
+    if (u == 0) return scale2c(exp(-a.lz[b].logn) * bp * es, kb + m - a.lz[b].k);
+    return scale2c(a.cU[ix] * bp * es, a.eU[ix] + kb + m);
+}
+
+__device__ __forceinline__ double seg_end_marg(const FbArgs &a, size_t rowbase, int u, int c)
+{
+    const size_t ix = (rowbase + u) * a.C + c;
+    return scale2c(a.cA[ix] * a.Vst[ix] * a.tIES[ix], a.eA[rowbase + u] + a.rbst[ix] - a.tM[ix]);
+}
+
+// Coverage mu[u,c] = sum_{s<=u} start(s,c) - sum_{1<=t<=u} end(t,c), a prefix scan
+// per (sequence, label) in chunks of covch positions (cov_chunk: about T/1024,
+// at least 32): chunk totals; their
+// exclusive prefix per (sequence, label), in order; the scan within each chunk
+// from that offset (writing raw mu into dX and the chunk's sum of mu); the
+// per-label sum over positions for the path through nu.
+__device__ __forceinline__ int cov_end(const FbArgs &a, int b, int u0)
+{
+    const int L = a.lengths[b];
+    return min(u0 + a.covch, (L >= 1 && L <= a.T) ? L : 0);
+}
+
+__global__ void cov_delta_kernel(FbArgs a)
+{
+    const int b = blockIdx.y, ch = blockIdx.x, c = threadIdx.x;
+    if (c >= a.C) return;
+    const int nch = (a.T + a.covch - 1) / a.covch;
+    const int u0 = ch * a.covch, u1 = cov_end(a, b, u0);
+    const size_t rowbase = (size_t)b * (a.T + 1);
+    double d0 = 0.0, d1 = 0.0;
+    int u = u0;
+    for (; u + 1 < u1; u += 2) {   // two independent positions per round
+        d0 += seg_start_marg(a, rowbase, b, u, c) - (u >= 1 ? seg_end_marg(a, rowbase, u, c) : 0.0);
+        d1 += seg_start_marg(a, rowbase, b, u + 1, c) - seg_end_marg(a, rowbase, u + 1, c);
+    }
+    if (u < u1) d0 += seg_start_marg(a, rowbase, b, u, c) - (u >= 1 ? seg_end_marg(a, rowbase, u, c) : 0.0);
+    a.covd[((size_t)b * nch + ch) * a.C + c] = d0 + d1;
+}
+
+// exclusive prefix of the chunk totals, in place, one thread per (sequence, label)
+__global__ void cov_offsets_kernel(FbArgs a)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= a.B * a.C) return;
+    const int b = i / a.C, c = i % a.C;
+    const int nch = (a.T + a.covch - 1) / a.covch;
+    double run = 0.0;
+    for (int k = 0; k < nch; ++k) {
+        double *p = &a.covd[((size_t)b * nch + k) * a.C + c];
+        const double d = *p;
+        *p = run;
+        run += d;
+    }
+}
+
+__global__ void cov_scan_kernel(FbArgs a)
+{
+    const int b = blockIdx.y, ch = blockIdx.x, c = threadIdx.x;
+    if (c >= a.C) return;
+    const int nch = (a.T + a.covch - 1) / a.covch;
+    const int u0 = ch * a.covch, u1 = cov_end(a, b, u0);
+    const size_t rowbase = (size_t)b * (a.T + 1);
+    double mu = a.covd[((size_t)b * nch + ch) * a.C + c];
+    double msum = 0.0;
+    for (int u = u0; u < u1; ++u) {
+        mu += seg_start_marg(a, rowbase, b, u, c) - (u >= 1 ? seg_end_marg(a, rowbase, u, c) : 0.0);
+        a.dX[((size_t)b * a.T + u) * a.C + c] = (float)mu;
+        msum += mu;
+    }
+    a.covm[((size_t)b * nch + ch) * a.C + c] = msum;
+}
+
+__global__ void cov_musum_kernel(FbArgs a)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= a.B * a.C) return;
+    const int b = i / a.C, c = i % a.C;
+    const int nch = (a.T + a.covch - 1) / a.covch;
+    double s = 0.0;
+    for (int k = 0; k < nch; ++k) s += a.covm[((size_t)b * nch + k) * a.C + c];
+    a.musum[(size_t)b * a.C + c] = s;
+}
 
 }  // namespace
 
@@ -204,10 +324,43 @@ void cl_grad_splits(int B, int T, int K, int C, int *nsD, int *nsA)
     const int tilesD = ceil_div(K, kTile) * ceil_div(C, kTile);
     const int tilesA = ceil_div(C, kTile) * ceil_div(C, kTile);
     long long d = ceil_div(4 * 148, tilesD), e = ceil_div(4 * 148, tilesA);
+    if (d > 1024) d = 1024;
+    if (e > 1024) e = 1024;
     *nsD = (int)(d < Q ? d : Q);
     *nsA = (int)(e < Q ? e : Q);
     if (*nsD < 1) *nsD = 1;
     if (*nsA < 1) *nsA = 1;
+}
+
+cudaError_t launch_rows_rescale(const FbArgs &a, cudaStream_t st)
+{
+    const size_t n = (size_t)a.B * (a.T + 1) * a.C;
+    int blocks = (int)((n + 255) / 256);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    prof_before(st);
+    rows_rescale<<<blocks, 256, 0, st>>>(a);
+    prof_after(st);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_coverage(const FbArgs &a, cudaStream_t st)
+{
+    const int nch = ceil_div(a.T, a.covch);
+    const int threads = ceil_div(a.C, 32) * 32;
+    const int nbc = ceil_div((long long)a.B * a.C, 128);
+    prof_before(st);
+    cov_delta_kernel<<<dim3(nch, a.B), threads, 0, st>>>(a);
+    prof_after(st);
+    prof_before(st);
+    cov_offsets_kernel<<<nbc, 128, 0, st>>>(a);
+    prof_after(st);
+    prof_before(st);
+    cov_scan_kernel<<<dim3(nch, a.B), threads, 0, st>>>(a);
+    prof_after(st);
+    prof_before(st);
+    cov_musum_kernel<<<nbc, 128, 0, st>>>(a);
+    prof_after(st);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_cl_param_grads(const FbArgs &a, cudaStream_t st)
@@ -218,9 +371,11 @@ cudaError_t launch_cl_param_grads(const FbArgs &a, cudaStream_t st)
     prof_before(st);
     trans_grad_kernel<<<dim3(a.nsA, ceil_div(a.C, kTile), ceil_div(a.C, kTile)), 256, 0, st>>>(a);
     prof_after(st);
-    const int n = a.C * a.C + a.K * a.C;
+    const int n = a.C * a.C + a.K * a.C;   // one warp per output
+    int blocks = ceil_div((long long)n * 32, 256);
+    if (blocks > 148 * 16) blocks = 148 * 16;
     prof_before(st);
-    cl_finalise_params<<<(n + 255) / 256, 256, 0, st>>>(a);
+    cl_finalise_params<<<blocks, 256, 0, st>>>(a);
     prof_after(st);
     return cudaGetLastError();
 }

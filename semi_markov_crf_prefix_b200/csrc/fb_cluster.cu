@@ -340,9 +340,16 @@ __device__ __forceinline__ bool wait_values(ClSmem &sm, int par, int u, bool ski
     }
 }
 
-template <int CPL, int MAXT, bool CLUSTER, bool RECOMPUTE>
-__global__ void __launch_bounds__(MAXT, 1) cl_fwd_kernel(FbArgs a, ClGeom g)
+// MODE 0: forward with checkpoints and log Z.  MODE 1: recompute one checkpoint
+// segment, writing the per-position rows relative to Z.  MODE 2: the whole
+// sequence once, log Z and the rows unscaled (scaled later by exp(-log Z)),
+// no checkpoints.  cid: the cluster's index among those running this body.
+template <int CPL, int MAXT, bool CLUSTER, int MODE>
+__device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, int cid)
 {
+    constexpr bool RECOMPUTE = MODE == 1;
+    constexpr bool ROWS = MODE != 0;
+    constexpr bool CKPT = MODE == 0;
     extern __shared__ __align__(16) double smc[];
     const int K = a.K, C = a.C, Cg = g.Cg, NT = g.NT, RS = g.RS, PW = g.PW;
     const int NOT = 32 * (g.NWO + g.NWT);   // owner + transition threads
@@ -350,7 +357,6 @@ __global__ void __launch_bounds__(MAXT, 1) cl_fwd_kernel(FbArgs a, ClGeom g)
     const int W0T = 32 * (g.NWO + g.NWT);   // first window thread
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rank = CLUSTER ? (int)cluster_rank() : 0;
-    const int cid = blockIdx.x / g.G;
     int b, seg;
     if constexpr (RECOMPUTE) {
         b = cid / a.J;
@@ -372,7 +378,7 @@ __global__ void __launch_bounds__(MAXT, 1) cl_fwd_kernel(FbArgs a, ClGeom g)
     const size_t rowbase = (size_t)b * (a.T + 1);
     unsigned char *ck_base = a.ckpt + ((size_t)b * a.J) * a.ckpt_stride;
     int kZ = 0;
-    double cz = 0.0;
+    double cz = MODE == 2 ? 1.0 : 0.0;
     if constexpr (RECOMPUTE) {
         kZ = a.lz[b].k;
         cz = exp(-a.lz[b].logn);
@@ -573,15 +579,15 @@ __global__ void __launch_bounds__(MAXT, 1) cl_fwd_kernel(FbArgs a, ClGeom g)
                     sm.ring[(tK + K) * RS + lc] = U;
                     U2 = U1;
                     U1 = U;
-                    if constexpr (RECOMPUTE) {
+                    if constexpr (ROWS) {
                         a.cU[row] = U * cz;
                         a.cA[row] = ap * cz;
                         a.eU[row] = r - kZ;
                     }
-                } else if constexpr (RECOMPUTE) {
+                } else if constexpr (ROWS) {
                     a.cA[row] = ap * cz;
                 }
-                if (RECOMPUTE && c == 0) a.eA[rowbase + t] = kt - kZ;
+                if (ROWS && c == 0) a.eA[rowbase + t] = kt - kZ;
                 f = f_n;
                 kt = kt_n;
             }
@@ -608,7 +614,7 @@ __global__ void __launch_bounds__(MAXT, 1) cl_fwd_kernel(FbArgs a, ClGeom g)
             if (ro.lab_ok && (j & 31) == 0) sm.pre3[((u + 2) & 3) * Cg * PW + lc * PW + (j >> 5)] = s;
         }
         if (cta_barrier_or(2, NT, timed_out)) timed_out = true;
-        if (!RECOMPUTE && td == 0 && t < L) {
+        if (CKPT && td == 0 && t < L) {
             // checkpoint t / delta: the ring at the reference of position t, r, k_{t+1}, k_{t+2}.
             // Row age 0 (row t) is there; ages 1..K-2 are at the reference of t-1; the
             // oldest row (age K-1, K >= 3) at that of t-2.
@@ -639,8 +645,18 @@ __global__ void __launch_bounds__(MAXT, 1) cl_fwd_kernel(FbArgs a, ClGeom g)
     if constexpr (CLUSTER) cluster_barrier();   // no CTA leaves while peers may still store to it
 }
 
-template <int CPL, int MAXT, bool CLUSTER>
-__global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
+template <int CPL, int MAXT, bool CLUSTER, bool RECOMPUTE>
+__global__ void __launch_bounds__(MAXT, 1) cl_fwd_kernel(FbArgs a, ClGeom g)
+{
+    cl_fwd_body<CPL, MAXT, CLUSTER, RECOMPUTE ? 1 : 0>(a, g, blockIdx.x / g.G);
+}
+
+// CHAIN = false: beta chain with the coverage marginal and dX on the chain, from
+// the recomputed forward rows.  CHAIN = true: the beta chain alone (it needs
+// nothing from the forward, so it can run beside it); the coverage is formed
+// later from the stored rows.  b: the sequence.
+template <int CPL, int MAXT, bool CLUSTER, bool CHAIN>
+__device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, int b)
 {
     extern __shared__ __align__(16) double smc[];
     const int K = a.K, C = a.C, Cg = g.Cg, NT = g.NT, RS = g.RS, PW = g.PW;
@@ -649,7 +665,6 @@ __global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
     const int W0T = 32 * (g.NWO + g.NWT);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rank = CLUSTER ? (int)cluster_rank() : 0;
-    const int b = blockIdx.x / g.G;
     const int L = a.lengths[b];
     if (L < 1 || L > a.T) {
         if (rank == 0 && tid == 0) set_status(a.status, SEMICRF_ERR_INVALID_LENGTH);
@@ -658,8 +673,8 @@ __global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
     const int c0l = rank * Cg, cg_own = min(Cg, C - c0l);
     ClSmem sm = cl_smem(smc, K, C, g, true);
     const size_t rowbase = (size_t)b * (a.T + 1);
-    const int kZ = a.lz[b].k;
-    const double cz = exp(-a.lz[b].logn);
+    const int kZ = CHAIN ? 0 : a.lz[b].k;   // the chain-only variant runs beside the forward
+    const double cz = CHAIN ? 0.0 : exp(-a.lz[b].logn);
     const Roles ro = cl_roles(g, warp, lane, c0l, cg_own);
     const int lc = ro.lc, j = ro.j, c = ro.c;
     const bool own = ro.is_own && ro.lab_ok;
@@ -713,7 +728,7 @@ __global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
             cp_async8(&sm.pf_es[sl * Cg + lc], a.tES + ix);
             cp_async8(&sm.pf_ies[sl * Cg + lc], a.tIES + ix);
             cp_async4(&sm.pf_m[sl * Cg + lc], a.tM + ix);
-            if (sp >= 1) {
+            if (!CHAIN && sp >= 1) {
                 cp_async8(&sm.pf_cu[sl * Cg + lc], a.cU + ix);
                 cp_async8(&sm.pf_ca[sl * Cg + lc], a.cA + ix);
                 cp_async4(&sm.pf_eu[sl * Cg + lc], a.eU + ix);
@@ -734,8 +749,14 @@ __global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
         const double eb = sm.pf_ies[sl * Cg + lc] * pow2c(rb - kb_o - m);   // exp(ln2 (rb - kb) - S)
         pbe_o = pre_o * eb;
         w0e_o = W0 * eb;
-        coef_o = (sn == 0) ? scale2c(cz, rb - kZ) : scale2c(sm.pf_cu[sl * Cg + lc], sm.pf_eu[sl * Cg + lc] + rb);
-        a2_o = (sn >= 1) ? scale2c(sm.pf_ca[sl * Cg + lc], sm.pf_ea[sl * Cg + lc] + kb_o) : 0.0;
+        if constexpr (!CHAIN) {
+            coef_o = (sn == 0) ? scale2c(cz, rb - kZ)
+                               : scale2c(sm.pf_cu[sl * Cg + lc], sm.pf_eu[sl * Cg + lc] + rb);
+            a2_o = (sn >= 1) ? scale2c(sm.pf_ca[sl * Cg + lc], sm.pf_ea[sl * Cg + lc] + kb_o) : 0.0;
+        } else {
+            coef_o = 0.0;
+            a2_o = 0.0;
+        }
     };
     if (own) {
         W0 = exp((double)a.D[c]);
@@ -746,7 +767,7 @@ __global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
         V1 = a.tES[(rowbase + L) * C + c];
         a.Vst[(rowbase + L) * C + c] = V1;
         a.rbst[(rowbase + L) * C + c] = rb;
-        mu_acc = scale2(a.cA[(rowbase + L) * C + c], a.eA[rowbase + L]);
+        mu_acc = CHAIN ? 0.0 : scale2(a.cA[(rowbase + L) * C + c], a.eA[rowbase + L]);
         for (int i = 1; i < kPF; ++i) prefetch(L - i);
         cp_async_wait<kPF - 2>();   // position L-1 has landed
         prepare(L - 1, 0, V2, pre, gg, pbe, w0e, coef, a2, kb);
@@ -813,9 +834,13 @@ __global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
                 // mu_acc holds the coverage of x[s] by label c; moving to x[s-1] adds the
                 // segments ending at s and removes those starting at s
                 const size_t row = (rowbase + s) * C + c;
-                if (a.dX) a.dX[((size_t)b * a.T + s) * C + c] = (float)mu_acc;
-                if (a.stst) a.stst[row] = start;
+                if constexpr (!CHAIN) {
+                    if (a.dX) a.dX[((size_t)b * a.T + s) * C + c] = (float)mu_acc;
+                    if (a.stst) a.stst[row] = start;
+                }
                 musum += mu_acc;
+                a.bpst[row] = bp;
+                if (c == 0) a.kbst[rowbase + s] = kb;
                 if (s >= 1) {
                     const double q = sm.qbuf[lc];
                     const double V = q * gg;
@@ -826,8 +851,6 @@ __global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
                     mu_acc += a2 * q - start;
                     a.Vst[row] = V;
                     a.rbst[row] = rb;
-                    a.bpst[row] = bp;
-                    if (c == 0) a.kbst[rowbase + s] = kb;
                 } else {
                     mu_acc -= start;
                 }
@@ -861,10 +884,28 @@ __global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
         sK = (sK == 0) ? K - 1 : sK - 1;
     }
     if (own) {
-        a.musum[(size_t)b * C + c] = musum;
-        a.mures[(size_t)b * C + c] = mu_acc;
+        if constexpr (!CHAIN) {
+            a.musum[(size_t)b * C + c] = musum;
+            a.mures[(size_t)b * C + c] = mu_acc;
+        }
     }
     if constexpr (CLUSTER) cluster_barrier();
+}
+
+template <int CPL, int MAXT, bool CLUSTER>
+__global__ void __launch_bounds__(MAXT, 1) cl_bwd_kernel(FbArgs a, ClGeom g)
+{
+    cl_bwd_body<CPL, MAXT, CLUSTER, false>(a, g, blockIdx.x / g.G);
+}
+
+// Forward (storing its rows) and the beta chain side by side: clusters [0, B)
+// run the forward of sequence b, clusters [B, 2B) the beta chain of b - B.
+template <int CPL, int MAXT, bool CLUSTER>
+__global__ void __launch_bounds__(MAXT, 1) cl_fused_kernel(FbArgs a, ClGeom g)
+{
+    const int cid = blockIdx.x / g.G;
+    if (cid < a.B) cl_fwd_body<CPL, MAXT, CLUSTER, 2>(a, g, cid);
+    else cl_bwd_body<CPL, MAXT, CLUSTER, true>(a, g, cid - a.B);
 }
 
 template <int CPL, int MAXT>
@@ -881,6 +922,41 @@ cudaError_t launch_cl_bwd_tpl(const ClGeom &g, const FbArgs &a, cudaStream_t st)
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)a.B * g.G);
+    cfg.blockDim = dim3(g.NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (cl) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = g.G;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    FbArgs aa = a;
+    ClGeom gg = g;
+    void *args[] = {&aa, &gg};
+    prof_before(st);
+    e = cudaLaunchKernelExC(&cfg, fn, args);
+    prof_after(st);
+    return e;
+}
+
+template <int CPL, int MAXT>
+cudaError_t launch_cl_fused_tpl(const ClGeom &g, const FbArgs &a, cudaStream_t st)
+{
+    const bool cl = g.G > 1;
+    void *fn = cl ? (void *)cl_fused_kernel<CPL, MAXT, true> : (void *)cl_fused_kernel<CPL, MAXT, false>;
+    const size_t smem = cl_smem_bytes_impl(a.K, a.C, g, true);   // the larger of the two layouts
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (g.G > 8) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2u * (unsigned)a.B * g.G);
     cfg.blockDim = dim3(g.NT);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
@@ -1063,6 +1139,17 @@ cudaError_t launch_cl_forward(const FbArgs &a, cudaStream_t st, bool recompute)
     if (!cl_plan(a.K, a.C, false, &g)) return cudaErrorInvalidConfiguration;
     const int cpl = cl_cpl_bucket(g.CPL), maxt = cl_max_threads(g.NT);
     SEMICRF_CL_TABLE(launch_cl_fwd_tpl, g, a, st, recompute)
+    return cudaErrorInvalidConfiguration;
+}
+
+// One geometry for both chains: the planner's backward plan (its layout is the
+// larger of the two and fits both).
+cudaError_t launch_cl_fused(const FbArgs &a, cudaStream_t st)
+{
+    ClGeom g;
+    if (!cl_plan(a.K, a.C, true, &g)) return cudaErrorInvalidConfiguration;
+    const int cpl = cl_cpl_bucket(g.CPL), maxt = cl_max_threads(g.NT);
+    SEMICRF_CL_TABLE(launch_cl_fused_tpl, g, a, st)
     return cudaErrorInvalidConfiguration;
 }
 

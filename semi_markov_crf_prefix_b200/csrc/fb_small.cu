@@ -112,24 +112,30 @@ __device__ __forceinline__ BwdSmem bwd_smem(double *base, int KM, int C)
 }
 
 // ===========================================================================
-// Forward (RECOMPUTE = false): one CTA per sequence, t = 1..L; checkpoint after
-// every delta-th step, log Z at t = L.  Recompute: one CTA per (sequence,
+// Forward, MODE 0: one CTA per sequence, t = 1..L; checkpoint after every
+// delta-th step, log Z at t = L.  MODE 1 (recompute): one CTA per (sequence,
 // checkpoint segment), replaying t = j*delta+1 .. min((j+1)*delta, L) and
-// writing the per-position forward quantities relative to Z.
+// writing the per-position forward quantities relative to Z.  MODE 2: the
+// whole sequence once, log Z, and the per-position quantities unscaled (the
+// caller applies exp(-log Z) once log Z is known); no checkpoints.
 // ===========================================================================
-template <int KM, int CM, bool RECOMPUTE>
-__global__ void __launch_bounds__(96) team_fwd_kernel(FbArgs a)
+template <int KM, int CM, int MODE>
+__device__ __forceinline__ void team_fwd_body(const FbArgs &a, int blk)
 {
+    constexpr bool RECOMPUTE = MODE == 1;
+    constexpr bool ROWS = MODE != 0;   // writes the per-position rows
+    constexpr bool CKPT = MODE == 0;   // writes checkpoints
     constexpr int NT = 96;
     extern __shared__ __align__(16) double smt[];
     const int K = a.K, C = a.C;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp >= 3) return;   // launched with a fourth warp alongside the backward
     int b, seg;
     if constexpr (RECOMPUTE) {
-        b = blockIdx.x / a.J;
-        seg = blockIdx.x % a.J;
+        b = blk / a.J;
+        seg = blk % a.J;
     } else {
-        b = blockIdx.x;
+        b = blk;
         seg = 0;
     }
     const int L = a.lengths[b];
@@ -148,7 +154,7 @@ __global__ void __launch_bounds__(96) team_fwd_kernel(FbArgs a)
     const size_t rowbase = (size_t)b * (a.T + 1);
     unsigned char *ck_base = a.ckpt + ((size_t)b * a.J) * a.ckpt_stride;
     int kZ = 0;
-    double c0 = 0.0;
+    double c0 = MODE == 2 ? 1.0 : 0.0;
     if constexpr (RECOMPUTE) {
         kZ = a.lz[b].k;
         c0 = exp(-a.lz[b].logn);
@@ -224,7 +230,8 @@ __global__ void __launch_bounds__(96) team_fwd_kernel(FbArgs a)
                         a.lz[b].k = k;
                         if (!isfinite(lz)) set_status(a.status, SEMICRF_ERR_DEVICE_RANGE);
                     }
-                } else {
+                }
+                if constexpr (ROWS) {
                     if (act) a.cA[(rowbase + t) * C + c] = ap * c0;
                     if (lane == 0) a.eA[rowbase + t] = k - kZ;
                 }
@@ -247,7 +254,7 @@ __global__ void __launch_bounds__(96) team_fwd_kernel(FbArgs a)
             }
             team_barrier(NT);
             if (__any_sync(0xffffffffu, sm.hbuf[par * 32 + lane] != 0)) team_barrier(NT);
-            if (!RECOMPUTE && td == 0 && t < L) team_barrier(NT);
+            if (CKPT && td == 0 && t < L) team_barrier(NT);
             tk = (tk + 1 == K) ? 0 : tk + 1;
             td = (td + 1 == a.delta) ? 0 : td + 1;
         }
@@ -325,7 +332,7 @@ __global__ void __launch_bounds__(96) team_fwd_kernel(FbArgs a)
                 }
                 team_barrier(NT);
             }
-            if (!RECOMPUTE && td == 0 && t < L) {
+            if (CKPT && td == 0 && t < L) {
                 // checkpoint t / delta: ring after step t, r, k_{t+1}
                 unsigned char *ck = ck_base + (size_t)(t / a.delta) * a.ckpt_stride;
                 double *ck_ring = reinterpret_cast<double *>(ck);
@@ -370,28 +377,37 @@ __global__ void __launch_bounds__(96) team_fwd_kernel(FbArgs a)
         for (int t = t_begin + 1; t <= t_end; ++t) {
             const int par = t & 1;
             prefetch(t + kP - 1);   // into the slot step t-1 used
-            if (RECOMPUTE && t - 1 > t_begin) write_out(t - 1);
+            if (ROWS && t - 1 > t_begin) write_out(t - 1);
             cp_async_wait<kP - 2>();   // step t+1 has landed
             team_barrier(NT);
             if (__any_sync(0xffffffffu, sm.hbuf[par * 32 + lane] != 0)) team_barrier(NT);
-            if (!RECOMPUTE && td == 0 && t < L) team_barrier(NT);
+            if (CKPT && td == 0 && t < L) team_barrier(NT);
             td = (td + 1 == a.delta) ? 0 : td + 1;
         }
-        if (RECOMPUTE && t_end < L) write_out(t_end);
+        if (ROWS && t_end < L) write_out(t_end);
     }
 }
 
+template <int KM, int CM, bool RECOMPUTE>
+__global__ void __launch_bounds__(96) team_fwd_kernel(FbArgs a)
+{
+    team_fwd_body<KM, CM, RECOMPUTE ? 1 : 0>(a, blockIdx.x);
+}
+
 // ===========================================================================
-// Backward: one CTA per sequence, s = L-1 .. 0.
+// Backward: one CTA per sequence, s = L-1 .. 0.  CHAIN = false: the marginals,
+// coverage and per-sequence dA, dD on the chain, from the recomputed forward
+// rows.  CHAIN = true: the beta chain only (it needs nothing from the forward,
+// so it can run beside it), storing per position V and its reference, the
+// normalised beta and the backward normaliser for the parallel passes.
 // ===========================================================================
-template <int KM, int CM>
-__global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
+template <int KM, int CM, bool CHAIN>
+__device__ __forceinline__ void team_bwd_body(const FbArgs &a, int b)
 {
     constexpr int NT = 128;
     extern __shared__ __align__(16) double smt[];
     const int K = a.K, C = a.C;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = blockIdx.x;
     const int L = a.lengths[b];
     if (L < 1 || L > a.T) {
         if (threadIdx.x == 0) set_status(a.status, SEMICRF_ERR_INVALID_LENGTH);
@@ -402,8 +418,8 @@ __global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
     BwdSmem sm = bwd_smem(smt, KM, C);
     double *col = sm.ring + (size_t)c * col_len(KM);   // row rho at (rho%K) and (rho%K)+K
     const size_t rowbase = (size_t)b * (a.T + 1);
-    const int kZ = a.lz[b].k;
-    const double c0 = exp(-a.lz[b].logn);
+    const int kZ = CHAIN ? 0 : a.lz[b].k;
+    const double c0 = CHAIN ? 0.0 : exp(-a.lz[b].logn);
 
     for (int i = threadIdx.x; i < 64; i += NT) {
         sm.xsh[i] = 0.0;
@@ -425,8 +441,12 @@ __global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
         const double W0 = act ? exp((double)a.D[c]) : 0.0;
         int rb = rb0, kb = 0;
         double Vprev = act ? a.tES[ixL] : 0.0;
-        double mu_acc = act ? scale2(a.cA[ixL], a.eA[rowbase + L]) : 0.0;
+        double mu_acc = (act && !CHAIN) ? scale2(a.cA[ixL], a.eA[rowbase + L]) : 0.0;
         double musum = 0.0;
+        if (CHAIN && act) {
+            a.Vst[ixL] = Vprev;
+            a.rbst[ixL] = rb;
+        }
         team_barrier(NT);
         team_barrier(NT);
         int sk = (L - 1) % K;   // s % K, kept incrementally
@@ -436,12 +456,19 @@ __global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
             const int m = sm.tM[slot * 32 + lane];
             double g = sm.tES[slot * 32 + lane] * pow2c(m + kb - rb);          // exp(S_s + ln2 (kb - rb))
             const double eb = sm.tIES[slot * 32 + lane] * pow2c(rb - kb - m);  // exp(ln2 (rb - kb) - S_s)
-            const double coef = (s == 0) ? scale2c(c0, rb - kZ)
-                                         : scale2c(sm.tCU[slot * 32 + lane], sm.tEU[slot * 32 + lane] + rb);
-            const double a2 = (s >= 1 && act) ? scale2c(sm.tCA[slot * 32 + lane], sm.tEA[slot] + kb) : 0.0;
+            double coef = 0.0, a2 = 0.0;
+            if constexpr (!CHAIN) {
+                coef = (s == 0) ? scale2c(c0, rb - kZ)
+                                : scale2c(sm.tCU[slot * 32 + lane], sm.tEU[slot * 32 + lane] + rb);
+                a2 = (s >= 1 && act) ? scale2c(sm.tCA[slot * 32 + lane], sm.tEA[slot] + kb) : 0.0;
+            }
             const double pb = fma(Vprev, W0, sm.prebuf[par * 32 + lane]);
             const double start = coef * pb;
             const double bp = pb * eb;
+            if (CHAIN && act) {
+                a.bpst[(rowbase + s) * C + c] = bp;
+                if (lane == 0) a.kbst[rowbase + s] = kb;
+            }
             const int ex = exponent_of(pb);
             const int h = (act && (ex > kRebaseBits || ex < -kRebaseBits)) ? -ex : 0;
             if (h != 0) {
@@ -472,8 +499,10 @@ __global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
                 n = 0.0;
                 for (int cc = 0; cc < C; ++cc) n += sm.xsh[par * 32 + cc];
             }
-            if (act && a.dX) a.dX[((size_t)b * a.T + s) * C + c] = (float)mu_acc;
-            if (act && a.stst) a.stst[(rowbase + s) * C + c] = start;
+            if constexpr (!CHAIN) {
+                if (act && a.dX) a.dX[((size_t)b * a.T + s) * C + c] = (float)mu_acc;
+                if (act && a.stst) a.stst[(rowbase + s) * C + c] = start;
+            }
             musum += mu_acc;
             if (s == 0) {
                 if (lane == 0) a.logzb[b] = kLn2 * (double)kb + log(n);
@@ -484,6 +513,10 @@ __global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
                 if (act) {
                     col[sk] = V;
                     col[sk + K] = V;
+                    if constexpr (CHAIN) {
+                        a.Vst[(rowbase + s) * C + c] = V;
+                        a.rbst[(rowbase + s) * C + c] = rb;
+                    }
                 }
                 mu_acc += a2 * q - start;
                 Vprev = V;
@@ -493,7 +526,7 @@ __global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
             if (__any_sync(0xffffffffu, sm.hbuf[par * 32 + lane] != 0)) team_barrier(NT);
             sk = (sk == 0) ? K - 1 : sk - 1;
         }
-        if (act) {
+        if (act && !CHAIN) {
             a.musum[(size_t)b * C + c] = musum;
             a.mures[(size_t)b * C + c] = mu_acc;
         }
@@ -521,22 +554,24 @@ __global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
             // Rows s+1 .. s+K-1 only: the chain overwrites row s+K's slot with row s
             // during this step.  They give the d = 1 dD term of position s and the
             // d = 2..K dD terms and duration sum of position s-1.
-            const double coef = (s == 0) ? scale2c(c0, rb - kZ)
-                                         : scale2c(sm.tCU[slot * 32 + lane], sm.tEU[slot * 32 + lane] + rb);
-            double coef_n = 0.0;
-            if (s >= 1) {
-                const int sn = (s - 1) & (kP - 1);
-                coef_n = (s - 1 == 0) ? scale2c(c0, rb - kZ)
-                                      : scale2c(sm.tCU[sn * 32 + lane], sm.tEU[sn * 32 + lane] + rb);
+            double coef = 0.0, coef_n = 0.0;
+            if constexpr (!CHAIN) {
+                coef = (s == 0) ? scale2c(c0, rb - kZ)
+                                : scale2c(sm.tCU[slot * 32 + lane], sm.tEU[slot * 32 + lane] + rb);
+                if (s >= 1) {
+                    const int sn = (s - 1) & (kP - 1);
+                    coef_n = (s - 1 == 0) ? scale2c(c0, rb - kZ)
+                                          : scale2c(sm.tCU[sn * 32 + lane], sm.tEU[sn * 32 + lane] + rb);
+                }
             }
             const double *base = col + sk1;   // base[j-1] is row s+j
-            accD[0] = fma(coef, base[0], accD[0]);
+            if constexpr (!CHAIN) accD[0] = fma(coef, base[0], accD[0]);
             double s0 = 0.0, s1 = 0.0;
 #pragma unroll
             for (int j = 1; j < KM; ++j) {
                 if (j < K) {
                     const double v = base[j - 1];
-                    accD[j] = fma(coef_n, v, accD[j]);
+                    if constexpr (!CHAIN) accD[j] = fma(coef_n, v, accD[j]);
                     if (j & 1) s1 = fma(v, W[j], s1);
                     else s0 = fma(v, W[j], s0);
                 }
@@ -560,7 +595,7 @@ __global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
             }
             sk1 = (sk1 == 0) ? K - 1 : sk1 - 1;
         }
-        if (act) {
+        if (act && !CHAIN) {
             double *accD_g = a.accD + (size_t)b * K * C;
 #pragma unroll
             for (int d = 0; d < KM; ++d)
@@ -575,7 +610,7 @@ __global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
         team_barrier(NT);
         for (int s = L - 1; s >= 0; --s) {
             const int par = s & 1;
-            if (s + 1 <= L - 1) {   // transition of position s+1: a2[s+1] outer b'[s+1]
+            if (!CHAIN && s + 1 <= L - 1) {   // transition of position s+1: a2[s+1] outer b'[s+1]
                 const int pp = (s + 1) & 1;
                 const double a2v = sm.a2buf[pp * 32 + lane];
 #pragma unroll
@@ -591,7 +626,7 @@ __global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
             team_barrier(NT);
             if (__any_sync(0xffffffffu, sm.hbuf[par * 32 + lane] != 0)) team_barrier(NT);
         }
-        if (act) {
+        if (act && !CHAIN) {
             double *accA_g = a.accA + (size_t)b * C * C + (size_t)c * C;
 #pragma unroll
             for (int cc = 0; cc < CM; ++cc)
@@ -606,7 +641,7 @@ __global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
                 cp_async8(&sm.tES[sl * 32 + lane], a.tES + ix);
                 cp_async8(&sm.tIES[sl * 32 + lane], a.tIES + ix);
                 cp_async4(&sm.tM[sl * 32 + lane], a.tM + ix);
-                if (sp >= 1) {
+                if (!CHAIN && sp >= 1) {
                     cp_async8(&sm.tCU[sl * 32 + lane], a.cU + ix);
                     cp_async8(&sm.tCA[sl * 32 + lane], a.cA + ix);
                     cp_async4(&sm.tEU[sl * 32 + lane], a.eU + ix);
@@ -632,14 +667,31 @@ __global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
 }
 
 template <int KM, int CM>
+__global__ void __launch_bounds__(128) team_bwd_kernel(FbArgs a)
+{
+    team_bwd_body<KM, CM, false>(a, blockIdx.x);
+}
+
+// Forward (storing its rows) and the beta chain side by side: blocks [0, B)
+// run the forward of sequence b, blocks [B, 2B) the beta chain of sequence b - B.
+template <int KM, int CM>
+__global__ void __launch_bounds__(128) team_fused_kernel(FbArgs a)
+{
+    if ((int)blockIdx.x < a.B) team_fwd_body<KM, CM, 2>(a, blockIdx.x);
+    else team_bwd_body<KM, CM, true>(a, blockIdx.x - a.B);
+}
+
+template <int KM, int CM>
 cudaError_t launch_team_tpl(const FbArgs &a, cudaStream_t st, int kind)
 {
-    const size_t smem = kind == 2 ? bwd_smem_bytes(KM, a.C) : fwd_smem_bytes(KM, a.C);
-    const unsigned grid = kind == 1 ? (unsigned)a.B * (unsigned)a.J : (unsigned)a.B;
-    const unsigned block = kind == 2 ? 128 : 96;
+    const size_t sf = fwd_smem_bytes(KM, a.C), sb = bwd_smem_bytes(KM, a.C);
+    const size_t smem = kind == 2 ? sb : kind == 3 ? (sf > sb ? sf : sb) : sf;
+    const unsigned grid = kind == 1 ? (unsigned)a.B * (unsigned)a.J : kind == 3 ? 2u * (unsigned)a.B : (unsigned)a.B;
+    const unsigned block = kind >= 2 ? 128 : 96;
     void *fn = kind == 0 ? (void *)team_fwd_kernel<KM, CM, false>
                : kind == 1 ? (void *)team_fwd_kernel<KM, CM, true>
-                           : (void *)team_bwd_kernel<KM, CM>;
+               : kind == 2 ? (void *)team_bwd_kernel<KM, CM>
+                           : (void *)team_fused_kernel<KM, CM>;
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     FbArgs aa = a;

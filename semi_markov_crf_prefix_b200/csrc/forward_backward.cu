@@ -195,4 +195,31 @@ cudaError_t launch_posteriors(const FbArgs &a0, float *mu, float *pstart, cudaSt
     return cudaGetLastError();
 }
 
+// Forward and backward at once: the forward chain (storing its rows unscaled, no
+// checkpoints) and the beta chain run side by side in one launch -- the beta
+// chain needs only S, A, D and the lengths -- then the rows get the log Z
+// scaling and the marginals, coverage and parameter gradients are parallel
+// passes over the stored rows.  11 launches.
+cudaError_t launch_forward_backward(const FbArgs &a, cudaStream_t st, int *launches)
+{
+    cudaError_t e = launch_exp_tables(a, st);
+    if (e != cudaSuccess) return e;
+    e = use_small(a.K, a.C) ? launch_small(a, st, 3) : launch_cl_fused(a, st);
+    if (e != cudaSuccess) return e;
+    e = launch_rows_rescale(a, st);
+    if (e != cudaSuccess) return e;
+    e = launch_coverage(a, st);
+    if (e != cudaSuccess) return e;
+    e = launch_cl_param_grads(a, st);
+    if (e != cudaSuccess) return e;
+    const size_t n = (size_t)a.B * a.T * a.C;
+    int blocks = (int)((n + 255) / 256);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    prof_before(st);
+    finalise_dx<<<blocks, 256, 0, st>>>(a);
+    prof_after(st);
+    *launches += 11;
+    return cudaGetLastError();
+}
+
 }  // namespace semicrf

@@ -129,6 +129,9 @@ bool make_layout(const semicrf_dims &d, int what, const Plan &p, Layout *out)
         L.gcA = take(B * C * C * 4);
         L.gcD = take(B * K * C * 4);
         L.gcN = take(B * C * 4);
+        const size_t nch = (T + cov_chunk(d.T) - 1) / cov_chunk(d.T);
+        L.covd = take(B * nch * C * 8);
+        L.covm = take(B * nch * C * 8);
         L.musum = take(B * C * 8);
         L.mures = take(B * C * 8);
         L.logzb = take(B * 8);
@@ -226,6 +229,9 @@ FbArgs fb_args(const semicrf_dims *d, const Layout &lay, void *ws)
     a.nsA = lay.nsA;
     a.partD = at<double>(ws, lay.partD);
     a.partA = at<double>(ws, lay.partA);
+    a.covd = at<double>(ws, lay.covd);
+    a.covm = at<double>(ws, lay.covm);
+    a.covch = cov_chunk(d->T);
     a.status = at<int32_t>(ws, lay.status);
     return a;
 }
@@ -310,6 +316,31 @@ semicrf_status semicrf_backward(const semicrf_dims *dims, const double *S, const
     a.dD = dD;
     int n = 0;
     cudaError_t e = launch_backward(p, a, static_cast<cudaStream_t>(stream), &n);
+    return finish(e, n);
+}
+
+semicrf_status semicrf_forward_backward(const semicrf_dims *dims, const double *S, const float *A,
+                                       const float *D, const int32_t *lengths, const double *grad_logZ,
+                                       void *ws, size_t ws_bytes, double *logZ, float *dX, double *dA,
+                                       double *dD, void *stream)
+{
+    Plan p;
+    Layout lay;
+    semicrf_status s = prepare(dims, SEMICRF_WS_TRAIN, ws, ws_bytes, &p, &lay);
+    if (s != SEMICRF_OK) return s;
+    if (!S || !A || !D || !lengths || !logZ || !dX || !dA || !dD) return SEMICRF_ERR_INVALID_ARG;
+    FbArgs a = fb_args(dims, lay, ws);
+    a.S = S;
+    a.A = A;
+    a.D = D;
+    a.lengths = lengths;
+    a.grad = grad_logZ;
+    a.logZ = logZ;
+    a.dX = dX;
+    a.dA = dA;
+    a.dD = dD;
+    int n = 0;
+    cudaError_t e = launch_forward_backward(a, static_cast<cudaStream_t>(stream), &n);
     return finish(e, n);
 }
 

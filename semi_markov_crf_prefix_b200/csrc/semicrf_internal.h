@@ -73,6 +73,8 @@ struct Layout {
     size_t gcA = 0;         // int32  [B][C][C]    gold transition counts
     size_t gcD = 0;         // int32  [B][K][C]    gold duration counts
     size_t gcN = 0;         // int32  [B][C]       gold positions per label
+    size_t covd = 0;        // double [B][ceil(T/cov_chunk(T))][C]  coverage chunk totals
+    size_t covm = 0;        // double [B][ceil(T/cov_chunk(T))][C]  coverage chunk sums over positions
     size_t musum = 0;       // double [B][C]
     size_t mures = 0;       // double [B][C]
     size_t logzb = 0;       // double [B]
@@ -122,6 +124,8 @@ struct FbArgs {
     int32_t *rbst, *kbst;
     int nsD, nsA;
     double *stst;   // when set, the backward stores the start marginals (posteriors)
+    double *covd, *covm;
+    int covch;
     float *dX;
     double *dA, *dD;
     int32_t *status;
@@ -140,13 +144,29 @@ struct ClGeom {
 bool cl_plan(int K, int C, bool bwd, ClGeom *out);
 cudaError_t launch_cl_forward(const FbArgs &a, cudaStream_t st, bool recompute);
 cudaError_t launch_cl_backward(const FbArgs &a, cudaStream_t st);
+// Forward storing its rows and the beta chain in one launch (2B clusters).
+cudaError_t launch_cl_fused(const FbArgs &a, cudaStream_t st);
 // dD and dA from the cluster backward's stored rows (cl_grads.cu): two contraction
 // kernels writing split partial sums, one kernel reducing them (3 launches).
 constexpr int kGradChunk = 64;   // start positions per staged chunk
 void cl_grad_splits(int B, int T, int K, int C, int *nsD, int *nsA);
 cudaError_t launch_cl_param_grads(const FbArgs &a, cudaStream_t st);
+// After the forward stored its rows unscaled (fused path): the recompute's scaling.
+cudaError_t launch_rows_rescale(const FbArgs &a, cudaStream_t st);
+// Coverage mu (raw, into dX) and its per-label sum (musum) from the stored rows (4 launches),
+// in chunks of cov_chunk(T) positions.
+inline int cov_chunk(int T)
+{
+    int ch = 32;
+    while ((long long)ch * 1024 < T) ch *= 2;
+    return ch;
+}
+cudaError_t launch_coverage(const FbArgs &a, cudaStream_t st);
+// Forward and backward chains side by side, then the parallel passes (fused path).
+cudaError_t launch_forward_backward(const FbArgs &a, cudaStream_t st, int *launches);
 
-// Warp-per-sequence kernels for C <= 32, K <= 32 (kind 0 forward, 1 recompute, 2 backward).
+// Warp-per-sequence kernels for C <= 32, K <= 32 (kind 0 forward, 1 recompute, 2 backward,
+// 3 forward storing its rows beside the beta chain).
 bool small_path_ok(int K, int C);
 cudaError_t launch_small(const FbArgs &a, cudaStream_t st, int kind);
 

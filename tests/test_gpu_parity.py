@@ -52,6 +52,32 @@ def run_gpu(w, ckpt_interval=0, grad=None, x=None, lengths=None):
                 vstatus=vstatus)
 
 
+def run_gpu_fused(w, grad=None):
+    """prefix_scan + forward_backward (both chains side by side) on cuda:0."""
+    torch = _torch()
+    import semi_markov_crf_prefix_b200 as sc
+    dev = torch.device("cuda:0")
+    xs = torch.from_numpy(np.ascontiguousarray(w.x)).to(dev)
+    A = torch.from_numpy(w.A).to(dev)
+    D = torch.from_numpy(w.D).to(dev)
+    lens = torch.from_numpy(np.ascontiguousarray(w.lengths)).to(dev)
+    g = None if grad is None else torch.from_numpy(np.asarray(grad, np.float64)).to(dev)
+    ws = sc.new_workspace(w.B, w.T, w.K, w.C, sc.WS_TRAIN, device=dev)
+    sc.clear_device_status(ws)
+    S, nu = sc.prefix_scan(xs, lens, ws=ws)
+    logZ, dX, dA, dD, _ = sc.forward_backward(S, A, D, lens, ws=ws, grad_logZ=g)
+    status = sc.device_status(ws)
+    wsv = sc.new_workspace(w.B, w.T, w.K, w.C, sc.WS_VITERBI, device=dev)
+    sc.clear_device_status(wsv)
+    score, labels, seg = sc.viterbi(S, A, D, lens, ws=wsv)
+    vstatus = sc.device_status(wsv)
+    torch.cuda.synchronize()
+    return dict(S=S.cpu().numpy(), nu=nu.cpu().numpy(), logZ=logZ.cpu().numpy(), dX=dX.cpu().numpy(),
+                dA=dA.cpu().numpy(), dD=dD.cpu().numpy(), score=score.cpu().numpy(),
+                labels=labels.cpu().numpy(), seg_start=seg.cpu().numpy(), status=status,
+                vstatus=vstatus)
+
+
 def check_against_oracle(w, g, grad=None, precision=True):
     o = oracle.factorised(w.x, w.A, w.D, w.lengths, grad_logZ=grad)
     assert g["status"] == 0 and g["vstatus"] == 0
@@ -262,3 +288,38 @@ def test_stress_million_positions():
     g2 = run_gpu(w2)
     lz = oracle.logz(w2.x, w2.A, w2.D, w2.lengths)
     assert g2["status"] == 0 and abs(g2["logZ"][0] - lz[0]) / abs(lz[0]) <= 1e-11
+
+
+
+# ------------------------------------------------------------------ fused path
+@pytest.mark.parametrize("name,path", [("tiny", None), ("ner", None), ("tiny", "general"), ("ner", "general")])
+def test_fused_named_small(name, path, monkeypatch):
+    if path:
+        monkeypatch.setenv("SEMICRF_KERNEL_PATH", path)
+    w = wl.make_workload(name)
+    grad = np.linspace(0.5, 1.5, w.B)
+    check_against_oracle(w, run_gpu_fused(w, grad=grad), grad=grad)
+
+
+@pytest.mark.parametrize("seed,B,T,K,C", [(8, 9, 90, 32, 32), (1, 5, 100, 1, 7), (4, 1, 1, 4, 5),
+                                           (5, 2, 50, 200, 9), (6, 3, 300, 40, 64), (7, 2, 200, 300, 20),
+                                           (2, 2, 70, 70, 2), (3, 4, 129, 33, 33)])
+def test_fused_random_shapes(seed, B, T, K, C):
+    w = wl.random_small(seed, B, T, K, C, ragged=True)
+    check_against_oracle(w, run_gpu_fused(w))
+
+
+def test_fused_large_workloads():
+    for w in (wl.make_workload("speech", B=4, T=1500), wl.make_workload("genomic", T=6000),
+              wl.make_workload("large", B=2, T=1500)):
+        check_against_oracle(w, run_gpu_fused(w))
+
+
+def test_fused_equals_checkpointed_path():
+    # the two ways of computing the same gradients agree to rounding
+    for w in (wl.make_workload("ner", B=8), wl.random_small(44, 3, 200, 40, 48, ragged=True)):
+        a, b = run_gpu(w), run_gpu_fused(w)
+        np.testing.assert_allclose(a["logZ"], b["logZ"], rtol=1e-14)
+        for k in ("dA", "dD"):
+            np.testing.assert_allclose(a[k], b[k], atol=1e-9, rtol=1e-11)
+        np.testing.assert_allclose(a["dX"], b["dX"], atol=2e-7, rtol=0)
