@@ -262,16 +262,22 @@ def run_gpu(args):
     for _ in range(args.steps):
         flush.zero_()                       # L2 flush between timed steps (not timed)
         t_start.record(stream)
-        step(profile=True)
+        step()
         t_end.record(stream)
         t_end.synchronize()
         step_ms.append(t_start.elapsed_time(t_end))
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    # per-kernel times: the same steps again, untimed, with events around every launch
+    for _ in range(args.steps):
+        flush.zero_()
+        step(profile=True)
+        torch.cuda.synchronize()
         for i, n in enumerate(KERNEL_NAMES):
             kern_ms[n] += evs[2 * i].elapsed_time(evs[2 * i + 1])
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    wall = time.perf_counter() - wall0
     total_ms = float(sum(step_ms))
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
