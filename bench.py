@@ -41,12 +41,14 @@ FP64_FMA_PER_SM_CLK = 64
 MUFU_PER_SM_CLK = 16
 HBM_FALLBACK_GBS = 6650.0
 SM_MAX_MHZ_FALLBACK = 1965.0
-# every kernel one step launches, in launch order: prefix_scan 3, then
-# forward_backward 11 (both chains side by side in one launch, then the passes
-# over the stored rows)
-SCAN_NAMES = ["scan_partials", "scan_offsets", "scan_apply"]
-FB_NAMES = ["exp_tables", "chains", "rows_rescale", "cov_delta", "cov_offsets", "cov_scan", "cov_musum",
-            "dur_grad", "trans_grad", "finalise_params", "finalise_dx"]
+# every kernel one step launches, in launch order, keyed by the launch count the
+# library reports: prefix_scan (1 launch for C <= 32 and T <= 2048, else 3), then
+# forward_backward (exp tables, both chains side by side in one launch, then
+# the passes over the stored rows: 2 for C, K <= 32, else 9)
+SCAN_NAMES = {1: ["prefix_scan"], 3: ["scan_partials", "scan_offsets", "scan_apply"]}
+FB_NAMES = {4: ["exp_tables", "chains", "post_rows", "post_finalise"],
+            11: ["exp_tables", "chains", "rows_rescale", "cov_delta", "cov_offsets", "cov_scan", "cov_musum",
+                 "dur_grad", "trans_grad", "finalise_params", "finalise_dx"]}
 
 
 def measured_peaks():
@@ -215,7 +217,12 @@ def run_gpu(args):
     dD = torch.empty((K, C), dtype=torch.float64, device=dev)
     flush = torch.empty(256 * 2**20 // 4, dtype=torch.float32, device=dev)
 
-    KERNEL_NAMES = SCAN_NAMES + FB_NAMES
+    # one untimed step to learn which kernels the path launches
+    sc.prefix_scan(x, lens, ws=ws, S=S, nu=nu)
+    scan_names = SCAN_NAMES[sc.last_launch_count()]
+    sc.forward_backward(S, A, D, lens, ws=ws, logZ=logZ, dX=dX, dA=dA, dD=dD)
+    fb_names = FB_NAMES[sc.last_launch_count()]
+    KERNEL_NAMES = scan_names + fb_names
     # per-kernel events (recorded by the library around each launch)
     n_ev = 2 * len(KERNEL_NAMES)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
@@ -226,10 +233,10 @@ def run_gpu(args):
 
     def step(profile=False):
         if profile:
-            lib.semicrf_set_profile_events(handles, 6)
+            lib.semicrf_set_profile_events(handles, 2 * len(scan_names))
         sc.prefix_scan(x, lens, ws=ws, S=S, nu=nu)
         if profile:
-            lib.semicrf_set_profile_events(ctypes_offset(handles, 6), 2 * len(FB_NAMES))
+            lib.semicrf_set_profile_events(ctypes_offset(handles, 2 * len(scan_names)), 2 * len(fb_names))
         sc.forward_backward(S, A, D, lens, ws=ws, logZ=logZ, dX=dX, dA=dA, dD=dD)
         if profile:
             lib.semicrf_set_profile_events(None, 0)

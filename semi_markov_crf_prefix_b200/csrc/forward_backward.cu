@@ -197,15 +197,22 @@ cudaError_t launch_posteriors(const FbArgs &a0, float *mu, float *pstart, cudaSt
 
 // Forward and backward at once: the forward chain (storing its rows unscaled, no
 // checkpoints) and the beta chain run side by side in one launch -- the beta
-// chain needs only S, A, D and the lengths -- then the rows get the log Z
-// scaling and the marginals, coverage and parameter gradients are parallel
-// passes over the stored rows.  11 launches.
+// chain needs only S, A, D and the lengths -- then the marginals, coverage and
+// parameter gradients are parallel passes over the stored rows: two launches
+// for C, K <= 32 (4 in all), else the rows get the log Z scaling and nine
+// launches follow (11 in all).
 cudaError_t launch_forward_backward(const FbArgs &a, cudaStream_t st, int *launches)
 {
     cudaError_t e = launch_exp_tables(a, st);
     if (e != cudaSuccess) return e;
-    e = use_small(a.K, a.C) ? launch_small(a, st, 3) : launch_cl_fused(a, st);
+    const bool small = use_small(a.K, a.C);
+    e = small ? launch_small(a, st, 3) : launch_cl_fused(a, st);
     if (e != cudaSuccess) return e;
+    if (small && a.npost > 0) {
+        e = launch_team_post(a, st);
+        if (e == cudaSuccess) *launches += 4;
+        return e;
+    }
     e = launch_rows_rescale(a, st);
     if (e != cudaSuccess) return e;
     e = launch_coverage(a, st);

@@ -123,15 +123,16 @@ bool make_layout(const semicrf_dims &d, int what, const Plan &p, Layout *out)
         L.bpst = take(B * (T + 1) * C * 8);
         L.kbst = take(B * (T + 1) * 4);
         cl_grad_splits(d.B, d.T, d.K, d.C, &L.nsD, &L.nsA);
-        L.partD = take((size_t)L.nsD * K * C * 8);
-        L.partA = take((size_t)L.nsA * C * C * 8);
+        L.npost = small_path_ok(d.K, d.C) ? team_post_splits(d.B, d.T) : 0;
+        L.partD = take((size_t)(L.nsD > L.npost ? L.nsD : L.npost) * K * C * 8);
+        L.partA = take((size_t)(L.nsA > L.npost ? L.nsA : L.npost) * C * C * 8);
         L.stst = take(B * (T + 1) * C * 8);
         L.gcA = take(B * C * C * 4);
         L.gcD = take(B * K * C * 4);
         L.gcN = take(B * C * 4);
         const size_t nch = (T + cov_chunk(d.T) - 1) / cov_chunk(d.T);
         L.covd = take(B * nch * C * 8);
-        L.covm = take(B * nch * C * 8);
+        L.covm = take(B * (size_t)team_post_chunks(d.T) * C * 8);   // cov_chunk >= 32: the larger count
         L.musum = take(B * C * 8);
         L.mures = take(B * C * 8);
         L.logzb = take(B * 8);
@@ -227,6 +228,7 @@ FbArgs fb_args(const semicrf_dims *d, const Layout &lay, void *ws)
     a.kbst = at<int32_t>(ws, lay.kbst);
     a.nsD = lay.nsD;
     a.nsA = lay.nsA;
+    a.npost = lay.npost;
     a.partD = at<double>(ws, lay.partD);
     a.partA = at<double>(ws, lay.partA);
     a.covd = at<double>(ws, lay.covd);

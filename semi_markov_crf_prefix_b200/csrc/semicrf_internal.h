@@ -67,14 +67,15 @@ struct Layout {
     size_t bpst = 0;        // double [B][T+1][C]
     size_t kbst = 0;        // int32  [B][T+1]
     int nsD = 0, nsA = 0;   // partial-sum splits of the dD and dA contractions
-    size_t partD = 0;       // double [nsD][K][C]
-    size_t partA = 0;       // double [nsA][C][C]
+    int npost = 0;          // CTAs of the C, K <= 32 post pass (team_post.cu), 0 otherwise
+    size_t partD = 0;       // double [max(nsD, npost)][K][C]
+    size_t partA = 0;       // double [max(nsA, npost)][C][C]
     size_t stst = 0;        // double [B][T+1][C]  P(segment of label c starts at s) (posteriors)
     size_t gcA = 0;         // int32  [B][C][C]    gold transition counts
     size_t gcD = 0;         // int32  [B][K][C]    gold duration counts
     size_t gcN = 0;         // int32  [B][C]       gold positions per label
     size_t covd = 0;        // double [B][ceil(T/cov_chunk(T))][C]  coverage chunk totals
-    size_t covm = 0;        // double [B][ceil(T/cov_chunk(T))][C]  coverage chunk sums over positions
+    size_t covm = 0;        // double [B][ceil(T/32)][C]  coverage chunk sums over positions
     size_t musum = 0;       // double [B][C]
     size_t mures = 0;       // double [B][C]
     size_t logzb = 0;       // double [B]
@@ -122,7 +123,7 @@ struct FbArgs {
     double *accD, *accA, *musum, *mures, *logzb;
     double *Vst, *bpst, *partD, *partA;
     int32_t *rbst, *kbst;
-    int nsD, nsA;
+    int nsD, nsA, npost;
     double *stst;   // when set, the backward stores the start marginals (posteriors)
     double *covd, *covm;
     int covch;
@@ -162,6 +163,11 @@ inline int cov_chunk(int T)
     return ch;
 }
 cudaError_t launch_coverage(const FbArgs &a, cudaStream_t st);
+// C, K <= 32: dD, dA, the coverage and dX from the stored rows in two launches
+// (team_post.cu): npost CTAs over (sequence, 32-position) items, then the finalise.
+int team_post_splits(int B, int T);
+int team_post_chunks(int T);
+cudaError_t launch_team_post(const FbArgs &a, cudaStream_t st);
 // Forward and backward chains side by side, then the parallel passes (fused path).
 cudaError_t launch_forward_backward(const FbArgs &a, cudaStream_t st, int *launches);
 

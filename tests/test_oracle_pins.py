@@ -364,6 +364,45 @@ def test_p9_viterbi(tiny10, tiny, ner):
             assert np.diff(np.append(starts, L)).max() <= w.K
 
 
+def test_p9_same_label_duration_swap_is_an_exact_tie(ner):
+    # Two adjacent segments of one label score the same in either order of their
+    # durations: the emission sums telescope to the same span and the same D and A
+    # terms appear.  So the best segmentation is not unique wherever it holds such
+    # a pair (the labels per position still are): brute force on a tiny problem
+    # finds several argmax segmentations with equal labels, and the definition
+    # scores the swapped segmentations of NER's Viterbi paths equal to rounding.
+    w = wl.random_small(3, 1, 6, 6, 1, ragged=False)   # one label: only durations differ
+    best, ties = -np.inf, []
+    for durs in bf.compositions(6, 6):
+        starts = np.zeros((1, 6), np.uint8)
+        starts[0, np.cumsum((0,) + durs[:-1])] = 1
+        sc = oracle.path_score(w.x, w.A, w.D, w.lengths, np.zeros((1, 6), np.int32), starts)[0]
+        if sc > best + 1e-12:
+            best, ties = sc, [starts]
+        elif abs(sc - best) <= 1e-12:
+            ties.append(starts)
+    durs = [tuple(np.diff(np.append(np.flatnonzero(t[0]), 6))) for t in ties]
+    assert all(sorted(d) == sorted(durs[0]) for d in durs)
+    assert len(ties) == math.factorial(len(durs[0])) // math.prod(
+        math.factorial(durs[0].count(v)) for v in set(durs[0]))
+    s, labels, seg = oracle.viterbi(ner.x, ner.A, ner.D, ner.lengths)
+    swapped = 0
+    for b in range(ner.B):
+        L = int(ner.lengths[b])
+        starts = list(np.flatnonzero(seg[b, :L])) + [L]
+        for i in range(len(starts) - 2):
+            a, m, e = starts[i], starts[i + 1], starts[i + 2]
+            if labels[b, a] == labels[b, m] and (m - a) != (e - m):
+                alt = seg.copy()
+                alt[b, m] = 0
+                alt[b, a + (e - m)] = 1
+                ps = oracle.path_score(ner.x[b:b + 1], ner.A, ner.D, ner.lengths[b:b + 1],
+                                       labels[b:b + 1], alt[b:b + 1])[0]
+                assert abs(ps - s[b]) <= 1e-12 * abs(s[b])
+                swapped += 1
+    assert swapped > 0
+
+
 # --------------------------------------------------------------------------- M8
 def test_m8_centring_controls_drift(ner):
     w = ner
