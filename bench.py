@@ -308,7 +308,14 @@ def run_gpu(args):
         h2d = hx.numel() * 4 + hA.numel() * 4 + hD.numel() * 4 + hl.numel() * 4
         d2h = h_logZ.numel() * 8 + h_dA.numel() * 8 + h_dD.numel() * 8
 
+        stage = sc.new_host_stage(B, T, K, C, device=dev)
+
         def e2e_step():
+            if world == 1:
+                # the C-ABI entry point for host buffers: copies in, scan, forward/backward, copies out
+                sc.forward_backward_host(hx, hA, hD, hl, ws, stage, logZ=h_logZ, dA=h_dA, dD=h_dD)
+                return
+            # several ranks: the parameter gradients are summed on the device before the copy out
             x.copy_(hx, non_blocking=True)
             A.copy_(hA, non_blocking=True)
             D.copy_(hD, non_blocking=True)

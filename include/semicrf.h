@@ -160,6 +160,29 @@ semicrf_status semicrf_forward_backward(const semicrf_dims *dims, const double *
                                        double *dD, void *stream);
 
 /*
+ * One forward/backward step from host memory, for callers whose inputs and
+ * results live on the host: copies x, A, D, lengths (and grad_logZ unless
+ * NULL) to the device, runs semicrf_prefix_scan and semicrf_forward_backward,
+ * and copies logZ, dA, dD (and dX unless dX is NULL) back, all on `stream`
+ * with one cudaMemcpyAsync per array.  Asynchronous: the host outputs hold the
+ * results once the stream has synchronised.  The host buffers should be pinned
+ * (cudaHostAlloc / cudaHostRegister) for the copies to run asynchronously;
+ * pageable buffers work, but then the copies block the calling thread.
+ * stage: caller-owned device memory of semicrf_host_stage_bytes(dims) bytes,
+ * 256-byte aligned, for the device copies, S and the device outputs (its
+ * regions: x, A, D, lengths, grad, S, nu, logZ, dX, dA, dD, each 256-byte
+ * aligned, so the results also stay readable there).  ws as for
+ * semicrf_forward_backward.  Errors: those of the two calls, plus
+ * SEMICRF_ERR_WORKSPACE_TOO_SMALL for a short stage and SEMICRF_ERR_CUDA for a
+ * failed copy.  semicrf_last_launch_count reports the kernels of both calls.
+ */
+size_t semicrf_host_stage_bytes(const semicrf_dims *dims);
+semicrf_status semicrf_forward_backward_host(const semicrf_dims *dims, const float *x, const float *A,
+                                            const float *D, const int32_t *lengths, const double *grad_logZ,
+                                            double *logZ, float *dX, double *dA, double *dD, void *stage,
+                                            size_t stage_bytes, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Viterbi: the forward recursion in (max, +), float64.  Ties pick the smallest
  * duration, then the smallest previous label; the final label is the smallest
  * reaching the maximum.  (The pages do not describe decoding; this follows the

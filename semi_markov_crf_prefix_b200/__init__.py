@@ -18,7 +18,8 @@ from . import _lib
 from ._lib import (MAX_C, MAX_K, WS_SCAN, WS_TRAIN, WS_VITERBI, SemiCRFError, dims,
                    status_string)
 
-__all__ = ["workspace_bytes", "new_workspace", "prefix_scan", "prefix_scan_noalloc", "forward", "backward",
+__all__ = ["workspace_bytes", "new_workspace", "new_host_stage", "forward_backward_host", "prefix_scan",
+           "prefix_scan_noalloc", "forward", "backward",
            "forward_backward", "viterbi",
            "posteriors", "gold_score", "gold_backward", "semicrf_nll",
            "logz_and_grads", "device_status", "clear_device_status", "last_launch_count",
@@ -186,6 +187,46 @@ def forward_backward(S, A, D, lengths, ws=None, grad_logZ=None, logZ=None, dX=No
                                                     _ptr(grad_logZ), _ptr(ws), ws.numel(), _ptr(logZ), _ptr(dX),
                                                     _ptr(dA), _ptr(dD), _stream(S.device)), "forward_backward")
     return logZ, dX, dA, dD, ws
+
+
+def new_host_stage(B, T, K, C, device="cuda"):
+    """Device staging buffer of forward_backward_host (uint8 tensor)."""
+    torch = _torch()
+    d = dims(B, T, K, C)
+    n = int(_lib.load().semicrf_host_stage_bytes(ctypes.byref(d)))
+    if n == 0:
+        raise ValueError("unsupported dimensions")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def forward_backward_host(x, A, D, lengths, ws, stage, grad_logZ=None, logZ=None, dA=None, dD=None, dX=None,
+                          want_dX=False):
+    """One step from host tensors (pin them for asynchronous copies): the library
+    copies x, A, D, lengths (and grad_logZ) to the device, runs prefix_scan and
+    forward_backward, and copies logZ, dA, dD (and dX when asked) back, all on the
+    current stream of the stage's device.  Returns (logZ, dA, dD, dX or None) as
+    host tensors, valid once that stream has synchronised."""
+    torch = _torch()
+    B, T, C = x.shape
+    K = D.shape[0]
+    for t, dt, shp, name in ((x, torch.float32, (B, T, C), "x"), (A, torch.float32, (C, C), "A"),
+                             (D, torch.float32, (K, C), "D"), (lengths, torch.int32, (B,), "lengths")):
+        if t.is_cuda or t.dtype != dt or tuple(t.shape) != shp or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous host {dt} tensor of shape {shp}")
+    if grad_logZ is not None and (grad_logZ.is_cuda or grad_logZ.dtype != torch.float64):
+        raise TypeError("grad_logZ must be a host float64 tensor")
+    pin = torch.cuda.is_available()
+    logZ = torch.empty(B, dtype=torch.float64, pin_memory=pin) if logZ is None else logZ
+    dA = torch.empty((C, C), dtype=torch.float64, pin_memory=pin) if dA is None else dA
+    dD = torch.empty((K, C), dtype=torch.float64, pin_memory=pin) if dD is None else dD
+    if want_dX and dX is None:
+        dX = torch.empty((B, T, C), dtype=torch.float32, pin_memory=pin)
+    d = dims(B, T, K, C)
+    _lib.check(_lib.load().semicrf_forward_backward_host(
+        ctypes.byref(d), _ptr(x), _ptr(A), _ptr(D), _ptr(lengths), _ptr(grad_logZ), _ptr(logZ), _ptr(dX),
+        _ptr(dA), _ptr(dD), _ptr(stage), stage.numel(), _ptr(ws), ws.numel(), _stream(stage.device)),
+        "forward_backward_host")
+    return logZ, dA, dD, dX
 
 
 def posteriors(S, A, D, lengths, ws, ckpt_interval=0, want_mu=True, want_pstart=True):

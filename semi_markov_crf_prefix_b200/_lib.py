@@ -54,6 +54,8 @@ SIGNATURES = {
     "semicrf_backward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P]),
     "semicrf_viterbi": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
     "semicrf_forward_backward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P, _P]),
+    "semicrf_host_stage_bytes": (ctypes.c_size_t, [_DP]),
+    "semicrf_forward_backward_host": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, _S, _P]),
     "semicrf_posteriors": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _S, _P, _P, _P]),
     "semicrf_gold_score": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
     "semicrf_gold_backward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),

@@ -346,6 +346,95 @@ semicrf_status semicrf_forward_backward(const semicrf_dims *dims, const double *
     return finish(e, n);
 }
 
+namespace {
+
+// Device staging of semicrf_forward_backward_host, in this order, each region
+// 256-byte aligned: x, A, D, lengths, grad, S, nu, logZ, dX, dA, dD.
+struct HostStage {
+    size_t x, A, D, len, grad, S, nu, logZ, dX, dA, dD, total;
+};
+
+HostStage host_stage_layout(const semicrf_dims &d)
+{
+    const size_t B = d.B, T = d.T, K = d.K, C = d.C;
+    HostStage h;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    h.x = take(B * T * C * 4);
+    h.A = take(C * C * 4);
+    h.D = take(K * C * 4);
+    h.len = take(B * 4);
+    h.grad = take(B * 8);
+    h.S = take(B * (T + 1) * C * 8);
+    h.nu = take(B * C * 8);
+    h.logZ = take(B * 8);
+    h.dX = take(B * T * C * 4);
+    h.dA = take(C * C * 8);
+    h.dD = take(K * C * 8);
+    h.total = off;
+    return h;
+}
+
+}  // namespace
+
+size_t semicrf_host_stage_bytes(const semicrf_dims *dims)
+{
+    if (check_dims_impl(dims) != SEMICRF_OK) return 0;
+    return host_stage_layout(*dims).total;
+}
+
+semicrf_status semicrf_forward_backward_host(const semicrf_dims *dims, const float *x, const float *A,
+                                            const float *D, const int32_t *lengths, const double *grad_logZ,
+                                            double *logZ, float *dX, double *dA, double *dD, void *stage,
+                                            size_t stage_bytes, void *ws, size_t ws_bytes, void *stream)
+{
+    semicrf_status s = check_dims_impl(dims);
+    if (s != SEMICRF_OK) return s;
+    if (!x || !A || !D || !lengths || !logZ || !dA || !dD || !stage) return SEMICRF_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(stage) % 256 != 0) return SEMICRF_ERR_INVALID_ARG;
+    const HostStage h = host_stage_layout(*dims);
+    if (stage_bytes < h.total) return SEMICRF_ERR_WORKSPACE_TOO_SMALL;
+    const size_t B = dims->B, T = dims->T, K = dims->K, C = dims->C;
+    char *st = static_cast<char *>(stage);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    auto h2d = [&](size_t off, const void *src, size_t bytes) {
+        return cudaMemcpyAsync(st + off, src, bytes, cudaMemcpyHostToDevice, cs);
+    };
+    cudaError_t e = h2d(h.x, x, B * T * C * 4);
+    if (e == cudaSuccess) e = h2d(h.A, A, C * C * 4);
+    if (e == cudaSuccess) e = h2d(h.D, D, K * C * 4);
+    if (e == cudaSuccess) e = h2d(h.len, lengths, B * 4);
+    if (e == cudaSuccess && grad_logZ) e = h2d(h.grad, grad_logZ, B * 8);
+    if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
+    s = semicrf_prefix_scan(dims, reinterpret_cast<const float *>(st + h.x),
+                            reinterpret_cast<const int32_t *>(st + h.len), reinterpret_cast<double *>(st + h.S),
+                            reinterpret_cast<double *>(st + h.nu), ws, ws_bytes, stream);
+    if (s != SEMICRF_OK) return s;
+    const int n_scan = g_last_launches;
+    s = semicrf_forward_backward(dims, reinterpret_cast<const double *>(st + h.S),
+                                 reinterpret_cast<const float *>(st + h.A), reinterpret_cast<const float *>(st + h.D),
+                                 reinterpret_cast<const int32_t *>(st + h.len),
+                                 grad_logZ ? reinterpret_cast<const double *>(st + h.grad) : nullptr, ws, ws_bytes,
+                                 reinterpret_cast<double *>(st + h.logZ), reinterpret_cast<float *>(st + h.dX),
+                                 reinterpret_cast<double *>(st + h.dA), reinterpret_cast<double *>(st + h.dD), stream);
+    if (s != SEMICRF_OK) return s;
+    const int n_fb = g_last_launches;
+    auto d2h = [&](void *dst, size_t off, size_t bytes) {
+        return cudaMemcpyAsync(dst, st + off, bytes, cudaMemcpyDeviceToHost, cs);
+    };
+    e = d2h(logZ, h.logZ, B * 8);
+    if (e == cudaSuccess) e = d2h(dA, h.dA, C * C * 8);
+    if (e == cudaSuccess) e = d2h(dD, h.dD, K * C * 8);
+    if (e == cudaSuccess && dX) e = d2h(dX, h.dX, B * T * C * 4);
+    if (e != cudaSuccess) return SEMICRF_ERR_CUDA;
+    g_last_launches = n_scan + n_fb;
+    return SEMICRF_OK;
+}
+
 semicrf_status semicrf_posteriors(const semicrf_dims *dims, const double *S, const float *A, const float *D,
                                   const int32_t *lengths, void *ws, size_t ws_bytes, float *mu, float *pstart,
                                   void *stream)

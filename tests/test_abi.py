@@ -98,6 +98,18 @@ def test_host_validation_before_launch(lib):
     # bad dims
     assert lib.semicrf_forward(_d(2, 64, 8, 300), fake, fake, fake, fake, fake, fake, tr, None) == \
         _lib.SEMICRF_ERR_UNSUPPORTED_SHAPE
+    # host-buffer step: stage sizing, short / null / misaligned stage, null host pointers
+    hs = lib.semicrf_host_stage_bytes(d)
+    assert hs > 0 and hs % 256 == 0 and lib.semicrf_host_stage_bytes(_d(0, 64, 8, 4)) == 0
+    fbh = lib.semicrf_forward_backward_host
+    assert fbh(d, fake, fake, fake, fake, None, fake, None, fake, fake, fake, hs - 1, fake, tr, None) == \
+        _lib.SEMICRF_ERR_WORKSPACE_TOO_SMALL
+    assert fbh(d, fake, fake, fake, fake, None, fake, None, fake, fake, None, hs, fake, tr, None) == \
+        _lib.SEMICRF_ERR_INVALID_ARG
+    assert fbh(d, fake, fake, fake, fake, None, fake, None, fake, fake, P((1 << 20) + 8), hs, fake, tr, None) == \
+        _lib.SEMICRF_ERR_INVALID_ARG
+    assert fbh(d, None, fake, fake, fake, None, fake, None, fake, fake, fake, hs, fake, tr, None) == \
+        _lib.SEMICRF_ERR_INVALID_ARG
     assert lib.semicrf_get_device_status(None, None) == _lib.SEMICRF_ERR_INVALID_ARG
     assert lib.semicrf_clear_device_status(None, None) == _lib.SEMICRF_ERR_INVALID_ARG
 

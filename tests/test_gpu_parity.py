@@ -351,6 +351,27 @@ def test_fused_rebased_columns(path, monkeypatch):
     check_against_oracle(w, run_gpu_fused(w, grad=grad), grad=grad)
 
 
+@pytest.mark.parametrize("name", ["ner", "tiny"])
+def test_host_buffer_step_equals_device_step(name):
+    # semicrf_forward_backward_host: the same kernels on the same inputs, so the
+    # same bits as prefix_scan + forward_backward on device tensors
+    torch = _torch()
+    import semi_markov_crf_prefix_b200 as sc
+    w = wl.make_workload(name)
+    grad = np.linspace(0.5, 1.5, w.B)
+    g = run_gpu_fused(w, grad=grad)
+    dev = torch.device("cuda:0")
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    ws = sc.new_workspace(w.B, w.T, w.K, w.C, sc.WS_TRAIN, device=dev)
+    stage = sc.new_host_stage(w.B, w.T, w.K, w.C, device=dev)
+    sc.clear_device_status(ws)
+    logZ, dA, dD, dX = sc.forward_backward_host(pin(w.x), pin(w.A), pin(w.D), pin(w.lengths), ws, stage,
+                                                grad_logZ=pin(grad), want_dX=True)
+    assert sc.device_status(ws) == 0   # synchronises the stream
+    for k, v in (("logZ", logZ), ("dA", dA), ("dD", dD), ("dX", dX)):
+        assert np.array_equal(v.numpy(), g[k]), k
+
+
 def test_fused_large_workloads():
     for w in (wl.make_workload("speech", B=4, T=1500), wl.make_workload("genomic", T=6000),
               wl.make_workload("large", B=2, T=1500)):
