@@ -12,8 +12,10 @@
 //   bp[s,c2]= the normalised backward score of a segment of label c2 starting at s
 // so X Y 2^(...) is the marginal of one segment (without exp D) and a2 bp the
 // marginal of one transition (without exp A).  The power-of-two factor is 1
-// unless the label's column was rebased between s+1 and s+d; a chunk checks that
-// once per label and takes the plain FMA path when it holds.
+// unless the label's column was rebased between s+1 and s+d; a chunk stages both
+// factors at one base reference per label (exact powers of two) so that every
+// term is one FMA, and falls back to exact per-term scaling for the whole CTA
+// only when a pre-scaled row would leave the safe range.
 //
 // Layout: each CTA owns a 32 x 32 tile of outputs ((d, c) or (c, c2)) and a
 // split z of the (sequence, 32-position chunk) list, which it walks chunk by
@@ -31,13 +33,17 @@ namespace {
 constexpr int kCh = 32;    // start positions per chunk
 constexpr int kTile = 32;  // output tile edge
 
+// Rows pre-scaled to a chunk's base reference are usable when none exceeds
+// 2^900: a product of two normal doubles is then exact to rounding, and where one
+// factor underflowed the product is below 2^-122 (negligible).
+__device__ __forceinline__ bool too_large(double v) { return !(fabs(v) <= 0x1p900); }
+
 __global__ void __launch_bounds__(256) dur_grad_kernel(FbArgs a)
 {
     __shared__ double xs[kCh][kTile];
     __shared__ int rs[kCh][kTile];
     __shared__ double ys[kCh + kTile][kTile];
     __shared__ int ry[kCh + kTile][kTile];
-    __shared__ int uni[kTile];
     const int K = a.K, C = a.C, T = a.T;
     const int z = blockIdx.x, c0 = blockIdx.y * kTile, d0 = 1 + blockIdx.z * kTile;   // d is 1-based
     const int tid = threadIdx.x, lc = tid & 31, dq = tid >> 5;
@@ -54,55 +60,56 @@ __global__ void __launch_bounds__(256) dur_grad_kernel(FbArgs a)
         const double g = a.grad ? a.grad[b] : 1.0;
         const int kZ = a.lz[b].k;
         const double cz = exp(-a.lz[b].logn);
+        const int tb = min(max(s0 + d0, 1), L);   // the chunk's base reference: rb at row tb
+        // Stage the chunk's start factors X (s in [s0, s0 + kCh), zero beyond L - 1)
+        // and end rows Y (t in [s0 + d0, s0 + d0 + kCh + kTile), zero beyond L).
+        // scaled: both at the label's base reference R0 (X 2^(R0 - rX), Y 2^(rY - R0)),
+        // so a segment marginal is one product; else at their own references.
+        auto stage = [&](bool scaled) {
+            bool bad = false;
+            for (int i = tid; i < kCh * kTile; i += 256) {
+                const int si = i / kTile, l2 = i % kTile, s = s0 + si, cc = c0 + l2;
+                double x = 0.0;
+                int r = INT_MIN;
+                if (s <= L - 1 && cc < C) {
+                    r = a.rbst[(rowbase + s + 1) * C + cc];
+                    x = (s == 0) ? scale2c(cz, r - kZ)
+                                 : scale2c(a.cU[(rowbase + s) * C + cc], a.eU[(rowbase + s) * C + cc] + r);
+                    x *= g;
+                    if (scaled) {
+                        x = scale2c(x, a.rbst[(rowbase + tb) * C + cc] - r);
+                        bad |= too_large(x);
+                    }
+                }
+                xs[si][l2] = x;
+                rs[si][l2] = r;
+            }
+            for (int i = tid; i < (kCh + kTile) * kTile; i += 256) {
+                const int ti = i / kTile, l2 = i % kTile, t = s0 + d0 + ti, cc = c0 + l2;
+                double y = 0.0;
+                int r = INT_MIN;
+                if (t <= L && cc < C) {
+                    y = a.Vst[(rowbase + t) * C + cc];
+                    r = a.rbst[(rowbase + t) * C + cc];
+                    if (scaled) {
+                        y = scale2c(y, r - a.rbst[(rowbase + tb) * C + cc]);
+                        bad |= too_large(y);
+                    }
+                }
+                ys[ti][l2] = y;
+                ry[ti][l2] = r;
+            }
+            return bad;
+        };
         __syncthreads();   // previous chunk's reads are done
-        // start factors X for s in [s0, s0 + kCh), zero beyond L - 1
-        for (int i = tid; i < kCh * kTile; i += 256) {
-            const int si = i / kTile, l2 = i % kTile, s = s0 + si, cc = c0 + l2;
-            double x = 0.0;
-            int r = INT_MIN;
-            if (s <= L - 1 && cc < C) {
-                r = a.rbst[(rowbase + s + 1) * C + cc];
-                x = (s == 0) ? scale2c(cz, r - kZ)
-                             : scale2c(a.cU[(rowbase + s) * C + cc], a.eU[(rowbase + s) * C + cc] + r);
-                x *= g;
-            }
-            xs[si][l2] = x;
-            rs[si][l2] = r;
+        // Extreme growth (a label's references over ~900 bits apart inside the
+        // chunk): the whole CTA restages at the own references and scales every term.
+        const bool exact = __syncthreads_or(stage(true));
+        if (exact) {
+            stage(false);
+            __syncthreads();
         }
-        // end rows V for t in [s0 + d0, s0 + d0 + kCh + kTile), zero beyond L
-        for (int i = tid; i < (kCh + kTile) * kTile; i += 256) {
-            const int ti = i / kTile, l2 = i % kTile, t = s0 + d0 + ti, cc = c0 + l2;
-            double y = 0.0;
-            int r = INT_MIN;
-            if (t <= L && cc < C) {
-                y = a.Vst[(rowbase + t) * C + cc];
-                r = a.rbst[(rowbase + t) * C + cc];
-            }
-            ys[ti][l2] = y;
-            ry[ti][l2] = r;
-        }
-        __syncthreads();
-        if (tid < kTile) {
-            // one reference for the whole chunk of this label?
-            int lo = INT_MAX, hi = INT_MIN;
-            for (int si = 0; si < kCh; ++si) {
-                const int r = rs[si][tid];
-                if (r != INT_MIN) {
-                    lo = min(lo, r);
-                    hi = max(hi, r);
-                }
-            }
-            for (int ti = 0; ti < kCh + kTile; ++ti) {
-                const int r = ry[ti][tid];
-                if (r != INT_MIN) {
-                    lo = min(lo, r);
-                    hi = max(hi, r);
-                }
-            }
-            uni[tid] = lo >= hi;
-        }
-        __syncthreads();
-        if (uni[lc]) {
+        if (!exact) {
 #pragma unroll 4
             for (int si = 0; si < kCh; ++si) {
                 const double x = xs[si][lc];
