@@ -1,9 +1,11 @@
 """Benchmark: semi-CRF forward+backward throughput on B200.
 
 One step = the whole hot path on one batch of synthetic input: centring and
-prefix scan, streaming forward (log Z + checkpoints), backward (checkpoint
-recompute, backward messages and marginals, gradient finalisation).  The
-metric is B*T*K*C segment-label updates per second (whole job over all ranks).
+prefix scan, then semicrf_forward_backward -- the forward chain (log Z, its
+per-position rows) and the backward chain side by side, then the marginals,
+coverage and gradient passes over the stored rows.  The metric is B*T*K*C
+segment-label updates per second (whole job over all ranks).  The end-to-end
+figure goes through semicrf_forward_backward_host (host buffers in and out).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config ner]
     python bench.py --impl reference ...   # the CPU oracle, same metric
