@@ -22,6 +22,7 @@
 // chunk, staging the chunk's rows in shared memory; it writes its tile of
 // partial sums to part*[z].  A last kernel adds the splits in order (the
 // result does not depend on scheduling) and applies exp(D), exp(A).
+#include <limits.h>
 #include <math.h>
 
 #include "device_util.cuh"
