@@ -6,6 +6,7 @@ The path computes in float64, so the tests also hold it to tighter internal
 bounds (marked "precision") that would catch a silent drop to float32.
 """
 import math
+import os
 
 import numpy as np
 import pytest
@@ -265,6 +266,25 @@ def test_zero_scores_closed_form_and_tie_break():
     np.testing.assert_allclose(g["logZ"][0], math.log(N[L]), rtol=1e-13)
     assert g["score"][0] == 0.0
     assert np.all(g["labels"][0] == 0) and np.all(g["seg_start"][0] == 1)
+
+
+def test_zero_scores_golden_at_workload_shapes():
+    # all-zero scores at the named workloads' K and C, lengths up to 5000 (both
+    # kernel families): log Z against the exact segmentation counts stored in
+    # tests/golden/zero_scores.txt; every Viterbi candidate ties at score 0
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "zero_scores.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    assert len(rows) >= 4
+    for L, K, C, z in rows:
+        L, K, C, z = int(L), int(K), int(C), float(z)
+        w = wl.random_small(0, 1, L, K, C, ragged=False)
+        w.x[:] = 0
+        w.A[:] = 0
+        w.D[:] = 0
+        g = run_gpu_fused(w)
+        assert g["status"] == 0 and g["vstatus"] == 0, (L, K, C)
+        np.testing.assert_allclose(g["logZ"][0], z, rtol=1e-12, err_msg=str((L, K, C)))
+        assert g["score"][0] == 0.0
 
 
 def test_genomic_full_size_invariants():

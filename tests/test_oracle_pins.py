@@ -20,6 +20,7 @@ transposed transition) fails at least one of them:
   M8  drift of the cumulative scores: centred << uncentred, S[L] = 0
 """
 import math
+import os
 
 import numpy as np
 import pytest
@@ -126,6 +127,25 @@ def test_p2_zero_scores_closed_form(L, K, C):
         np.testing.assert_allclose(f["dA"], np.full((C, C), (L - 1) / (C * (1 + C))), rtol=1e-11)
         # coverage is uniform over labels
         np.testing.assert_allclose(f["dX"], 0.0, atol=1e-13)
+
+
+def _golden_zero_scores():
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "zero_scores.txt")
+    rows = [l.split() for l in open(path) if l.strip() and not l.startswith("#")]
+    return [(int(L), int(K), int(C), float(z)) for L, K, C, z in rows]
+
+
+def test_p2_golden_zero_scores_fixture():
+    # the stored closed-form values (exact integer counts) against the oracle,
+    # at the shapes the oracle finishes quickly
+    rows = _golden_zero_scores()
+    assert len(rows) >= 4
+    for L, K, C, z in rows:
+        if L * (K * C + C * C) > 2e7:
+            continue
+        assert math.isclose(math.log(_zero_counts(L, K, C)), z, rel_tol=1e-15)
+        f = oracle.factorised(np.zeros((1, L, C)), np.zeros((C, C)), np.zeros((K, C)), np.array([L], np.int32))
+        np.testing.assert_allclose(f["logZ"][0], z, rtol=1e-13)
 
 
 def test_p2_viterbi_tie_break_on_zeros():
