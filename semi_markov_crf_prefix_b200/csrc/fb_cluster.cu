@@ -1018,20 +1018,6 @@ cudaError_t launch_cl_fwd_tpl(const ClGeom &g, const FbArgs &a, cudaStream_t st,
 int cl_max_threads(int nt) { return nt <= 256 ? 256 : nt <= 512 ? 512 : nt <= 768 ? 768 : 1024; }
 int cl_cpl_bucket(int cpl) { return cpl <= 4 ? 4 : cpl <= 8 ? 8 : cpl <= 16 ? 16 : 32; }
 
-int pow2_floor(int v)
-{
-    int p = 1;
-    while (p * 2 <= v) p *= 2;
-    return p;
-}
-
-int pow2_ceil(int v)
-{
-    int p = 1;
-    while (p < v) p *= 2;
-    return p;
-}
-
 }  // namespace
 
 // One candidate geometry: G CTAs, LPL transition lanes per label, LPW window
