@@ -113,9 +113,13 @@ semicrf_status semicrf_prefix_scan(const semicrf_dims *dims, const float *x,
  * every GPU that loads the library until exit; requires B*C <= 131072
  * (SEMICRF_ERR_UNSUPPORTED_SHAPE otherwise).  Allocates nothing.  The first call
  * on a device looks up the array's device address (make it before any stream
- * capture).  All calls share the array: calls that overlap on the GPU race and
- * must be serialised by the caller.  Device-side length errors are not
- * reported by this entry point (such sequences are skipped).
+ * capture) and keeps it for the life of the process, so after cudaDeviceReset
+ * on a device this entry point must not be called on that device again.  All
+ * calls share the array: calls issued in order on one stream are safe; calls
+ * that can overlap on the GPU (different streams, or host threads without an
+ * ordering between their streams) race and must be serialised by the caller.
+ * Device-side length errors are not reported by this entry point (such
+ * sequences are skipped).
  */
 semicrf_status semicrf_prefix_scan_noalloc(const semicrf_dims *dims, const float *x,
                                            const int32_t *lengths, double *S, double *nu,
@@ -240,6 +244,28 @@ semicrf_status semicrf_gold_backward(const semicrf_dims *dims, const int32_t *le
                                      const double *grad_score, float *dX, double *dA, double *dD,
                                      void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * Training objective (technical summary section 3: training by negative
+ * log-likelihood): nll[b] = log Z_b - score_b(y*) for the gold segmentations
+ * given as for semicrf_gold_score.  Runs semicrf_forward (log Z into logZ, the
+ * checkpoints into ws) and the gold score (into score), and forms nll on the
+ * device.  Errors and device findings as for those two calls.
+ */
+semicrf_status semicrf_nll(const semicrf_dims *dims, const double *S, const float *A, const float *D,
+                           const int32_t *lengths, const int32_t *labels, const uint8_t *seg_start,
+                           double *logZ, double *score, double *nll, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Gradient of sum_b g_b nll[b] (g = grad_nll, NULL: ones) with respect to the
+ * emissions (through S and nu), A and D, OVERWRITING dX, dA, dD: semicrf_backward
+ * with weights g, then the gold-segmentation counts with weights -g.  ws must be
+ * the workspace of the matching semicrf_nll call.
+ */
+semicrf_status semicrf_nll_backward(const semicrf_dims *dims, const double *S, const float *A, const float *D,
+                                    const int32_t *lengths, const int32_t *labels, const uint8_t *seg_start,
+                                    const double *grad_nll, void *ws, size_t ws_bytes, float *dX, double *dA,
+                                    double *dD, void *stream);
+
 /* Zero the device status word in ws (asynchronous on stream). */
 semicrf_status semicrf_clear_device_status(void *ws, void *stream);
 
@@ -251,6 +277,24 @@ semicrf_status semicrf_get_device_status(const void *ws, void *stream);
 
 /* Static, human-readable name of a status. */
 const char *semicrf_status_string(semicrf_status s);
+
+/*
+ * Launch geometry of the sequential chains for these dims, for tuning and
+ * diagnostics (no counterpart on the pages).  path: 0 the forward_backward
+ * step (forward and backward chains in one launch), 1 semicrf_forward,
+ * 2 semicrf_backward.  Fills info[0..8] (n >= 9):
+ *   info[0]  kernel family: 0 = one CTA per sequence (C <= 32 and K <= 32),
+ *            1 = one thread-block cluster per chain
+ *   info[1]  CTAs per cluster G      info[2] threads per CTA
+ *   info[3]  labels per CTA          info[4] transition lanes per label
+ *   info[5]  window lanes per label  info[6] dynamic shared memory per CTA (bytes)
+ *   info[7]  clusters of this shape the current device can hold at once
+ *            (-1 when not queried or when the CUDA query fails)
+ *   info[8]  clusters the launch needs (2B for path 0, else B)
+ * Family 0 fills info[0], info[1] = 1, info[7] = -1 and info[8] only.  Host
+ * only, except the occupancy query (a CUDA runtime call, no launch).
+ */
+semicrf_status semicrf_chain_plan(const semicrf_dims *dims, int32_t path, int32_t *info, int32_t n);
 
 /* Kernel launches issued by the most recent successful call on this thread. */
 int32_t semicrf_last_launch_count(void);

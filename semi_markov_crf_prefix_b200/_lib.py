@@ -59,10 +59,13 @@ SIGNATURES = {
     "semicrf_posteriors": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _S, _P, _P, _P]),
     "semicrf_gold_score": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
     "semicrf_gold_backward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "semicrf_nll": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "semicrf_nll_backward": (ctypes.c_int, [_DP, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, _P, _P, _P]),
     "semicrf_clear_device_status": (ctypes.c_int, [_P, _P]),
     "semicrf_get_device_status": (ctypes.c_int, [_P, _P]),
     "semicrf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "semicrf_last_launch_count": (ctypes.c_int32, []),
+    "semicrf_chain_plan": (ctypes.c_int, [_DP, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]),
     "semicrf_set_profile_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]),
 }
 

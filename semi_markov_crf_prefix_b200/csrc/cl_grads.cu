@@ -331,7 +331,8 @@ void cl_grad_splits(int B, int T, int K, int C, int *nsD, int *nsA)
     const long long Q = (long long)B * ceil_div(T, kCh);
     const int tilesD = ceil_div(K, kTile) * ceil_div(C, kTile);
     const int tilesA = ceil_div(C, kTile) * ceil_div(C, kTile);
-    long long d = ceil_div(4 * 148, tilesD), e = ceil_div(4 * 148, tilesA);
+    const int nsm = device_sm_count();
+    long long d = ceil_div(4 * nsm, tilesD), e = ceil_div(4 * nsm, tilesA);
     if (d > 1024) d = 1024;
     if (e > 1024) e = 1024;
     *nsD = (int)(d < Q ? d : Q);
@@ -344,7 +345,7 @@ cudaError_t launch_rows_rescale(const FbArgs &a, cudaStream_t st)
 {
     const size_t n = (size_t)a.B * (a.T + 1) * a.C;
     int blocks = (int)((n + 255) / 256);
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks > device_sm_count() * 16) blocks = device_sm_count() * 16;
     prof_before(st);
     rows_rescale<<<blocks, 256, 0, st>>>(a);
     prof_after(st);
@@ -381,7 +382,7 @@ cudaError_t launch_cl_param_grads(const FbArgs &a, cudaStream_t st)
     prof_after(st);
     const int n = a.C * a.C + a.K * a.C;   // one warp per output
     int blocks = ceil_div((long long)n * 32, 256);
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks > device_sm_count() * 16) blocks = device_sm_count() * 16;
     prof_before(st);
     cl_finalise_params<<<blocks, 256, 0, st>>>(a);
     prof_after(st);

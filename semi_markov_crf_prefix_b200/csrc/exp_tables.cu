@@ -33,7 +33,7 @@ cudaError_t launch_exp_tables(const FbArgs &a, cudaStream_t st)
 {
     const size_t n = (size_t)a.B * (a.T + 1) * a.C;
     int blocks = (int)((n + 255) / 256);
-    if (blocks > 148 * 8) blocks = 148 * 8;
+    if (blocks > device_sm_count() * 8) blocks = device_sm_count() * 8;
     prof_before(st);
     exp_tables_kernel<<<blocks, 256, 0, st>>>(a);
     prof_after(st);

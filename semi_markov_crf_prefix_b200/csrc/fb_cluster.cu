@@ -1015,6 +1015,45 @@ cudaError_t launch_cl_fwd_tpl(const ClGeom &g, const FbArgs &a, cudaStream_t st,
     return e;
 }
 
+// How many clusters of this geometry the GPU can hold at once (path 0: the fused
+// launch, 1: the forward, 2: the backward); G = 1 counts CTAs.
+template <int CPL, int MAXT>
+cudaError_t occ_cl_tpl(const ClGeom &g, int K, int C, int path, int *nclusters)
+{
+    const bool cl = g.G > 1;
+    void *fn;
+    if (path == 0) fn = cl ? (void *)cl_fused_kernel<CPL, MAXT, true> : (void *)cl_fused_kernel<CPL, MAXT, false>;
+    else if (path == 1) fn = cl ? (void *)cl_fwd_kernel<CPL, MAXT, true, false> : (void *)cl_fwd_kernel<CPL, MAXT, false, false>;
+    else fn = cl ? (void *)cl_bwd_kernel<CPL, MAXT, true> : (void *)cl_bwd_kernel<CPL, MAXT, false>;
+    const size_t smem = cl_smem_bytes_impl(K, C, g, path != 1);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (g.G > 8) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    if (!cl) {
+        int nb = 0, dev = 0, nsm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, g.NT, smem);
+        if (e == cudaSuccess) e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+        *nclusters = nb * nsm;
+        return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)g.G);
+    cfg.blockDim = dim3(g.NT);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = g.G;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaOccupancyMaxActiveClusters(nclusters, fn, &cfg);
+}
+
 int cl_max_threads(int nt) { return nt <= 256 ? 256 : nt <= 512 ? 512 : nt <= 768 ? 768 : 1024; }
 int cl_cpl_bucket(int cpl) { return cpl <= 4 ? 4 : cpl <= 8 ? 8 : cpl <= 16 ? 16 : 32; }
 
@@ -1148,6 +1187,37 @@ cudaError_t launch_cl_backward(const FbArgs &a, cudaStream_t st)
     return cudaErrorInvalidConfiguration;
 }
 #undef SEMICRF_CL_TABLE
+
+// The geometry the planner picks for a path and how many such clusters fit at
+// once: info = {G, NT, Cg, LPL, LPW, shared bytes, resident clusters (-1 when the
+// CUDA query fails, e.g. without a GPU)}.
+bool cl_plan_info(int K, int C, int path, int32_t *info)
+{
+    ClGeom g;
+    if (!cl_plan(K, C, path != 1, &g)) return false;
+    info[0] = g.G;
+    info[1] = g.NT;
+    info[2] = g.Cg;
+    info[3] = g.LPL;
+    info[4] = g.LPW;
+    info[5] = (int32_t)cl_smem_bytes_impl(K, C, g, path != 1);
+    info[6] = -1;
+    const int cpl = cl_cpl_bucket(g.CPL), maxt = cl_max_threads(g.NT);
+    int n = -1;
+    cudaError_t e = cudaErrorInvalidConfiguration;
+#define SEMICRF_OCC_CASE(CPL, MAXT) \
+    if (cpl == CPL && maxt == MAXT) e = occ_cl_tpl<CPL, MAXT>(g, K, C, path, &n)
+    SEMICRF_OCC_CASE(4, 256); SEMICRF_OCC_CASE(4, 512); SEMICRF_OCC_CASE(4, 768); SEMICRF_OCC_CASE(4, 1024);
+    SEMICRF_OCC_CASE(8, 256); SEMICRF_OCC_CASE(8, 512); SEMICRF_OCC_CASE(8, 768); SEMICRF_OCC_CASE(8, 1024);
+    SEMICRF_OCC_CASE(16, 256); SEMICRF_OCC_CASE(16, 512); SEMICRF_OCC_CASE(16, 768);
+    SEMICRF_OCC_CASE(32, 256); SEMICRF_OCC_CASE(32, 512);
+#undef SEMICRF_OCC_CASE
+    if (e == cudaSuccess) info[6] = n;
+    else cudaGetLastError();   // clear a failed query
+    return true;
+}
+
+
 #undef SEMICRF_CL_CASE
 
 }  // namespace semicrf

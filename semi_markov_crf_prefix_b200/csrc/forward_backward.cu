@@ -167,7 +167,7 @@ cudaError_t launch_backward(const Plan &p, const FbArgs &a, cudaStream_t st, int
     }
     const size_t n = (size_t)a.B * a.T * a.C;
     int blocks = (int)((n + 255) / 256);
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks > device_sm_count() * 16) blocks = device_sm_count() * 16;
     prof_before(st);
     finalise_dx<<<blocks, 256, 0, st>>>(a);
     prof_after(st);
@@ -186,7 +186,7 @@ cudaError_t launch_posteriors(const FbArgs &a0, float *mu, float *pstart, cudaSt
     if (e != cudaSuccess) return e;
     const size_t n = (mu ? (size_t)a.B * a.T * a.C : 0) + (pstart ? (size_t)a.B * a.T : 0);
     int blocks = (int)((n + 255) / 256);
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks > device_sm_count() * 16) blocks = device_sm_count() * 16;
     if (blocks < 1) blocks = 1;
     prof_before(st);
     posterior_finalise<<<blocks, 256, 0, st>>>(a, mu, pstart);
@@ -221,7 +221,7 @@ cudaError_t launch_forward_backward(const FbArgs &a, cudaStream_t st, int *launc
     if (e != cudaSuccess) return e;
     const size_t n = (size_t)a.B * a.T * a.C;
     int blocks = (int)((n + 255) / 256);
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks > device_sm_count() * 16) blocks = device_sm_count() * 16;
     prof_before(st);
     finalise_dx<<<blocks, 256, 0, st>>>(a);
     prof_after(st);

@@ -19,6 +19,12 @@ namespace {
 
 constexpr int kGoldThreads = 256;
 
+// Weight of sequence b in the gradient: wsign * g_b (g_b = 1 without weights).
+__device__ __forceinline__ double gold_weight(const GoldArgs &a, int b)
+{
+    return a.wsign * (a.grad ? a.grad[b] : 1.0);
+}
+
 // End of the segment starting at s, or -1 if the segmentation is malformed there.
 __device__ __forceinline__ int gold_segment_end(const GoldArgs &a, size_t pb, int s, int L, int c)
 {
@@ -73,6 +79,7 @@ __global__ void __launch_bounds__(kGoldThreads) gold_score_kernel(GoldArgs a)
     if (tid == 0) {
         if (!ok_len) set_status(a.status, SEMICRF_ERR_INVALID_LENGTH);
         a.score[b] = part[0];
+        if (a.nll) a.nll[b] = a.logZ[b] - part[0];
     }
     if (bad) set_status(a.status, SEMICRF_ERR_INVALID_SEGMENTATION);
 }
@@ -120,11 +127,11 @@ __global__ void gold_param_kernel(GoldArgs a)
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nA + nD; i += gridDim.x * blockDim.x) {
         double s = 0.0;
         if (i < nA) {
-            for (int b = 0; b < a.B; ++b) s += (a.grad ? a.grad[b] : 1.0) * (double)a.cntA[(size_t)b * nA + i];
+            for (int b = 0; b < a.B; ++b) s += gold_weight(a, b) * (double)a.cntA[(size_t)b * nA + i];
             a.dA[i] += s;
         } else {
             const int k = i - nA;
-            for (int b = 0; b < a.B; ++b) s += (a.grad ? a.grad[b] : 1.0) * (double)a.cntD[(size_t)b * nD + k];
+            for (int b = 0; b < a.B; ++b) s += gold_weight(a, b) * (double)a.cntD[(size_t)b * nD + k];
             a.dD[k] += s;
         }
     }
@@ -141,7 +148,7 @@ __global__ void gold_dx_kernel(GoldArgs a)
         const int b = (int)(bt / a.T);
         const int L = a.lengths[b];
         if (L < 1 || L > a.T || u >= L) continue;
-        const double g = a.grad ? a.grad[b] : 1.0;
+        const double g = gold_weight(a, b);
         const double ind = a.labels[bt] == c ? 1.0 : 0.0;
         const double mean = (double)a.cntN[(size_t)b * a.C + c] / (double)L;
         a.dX[i] = (float)((double)a.dX[i] + g * (ind - mean));
@@ -170,7 +177,7 @@ cudaError_t launch_gold_backward(const GoldArgs &a, cudaStream_t st, int *launch
     prof_after(st);
     const size_t n = (size_t)a.B * a.T * a.C;
     int blocks = (int)((n + 255) / 256);
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks > device_sm_count() * 16) blocks = device_sm_count() * 16;
     prof_before(st);
     gold_dx_kernel<<<blocks, 256, 0, st>>>(a);
     prof_after(st);

@@ -14,9 +14,12 @@
 // process exits.  Host code cannot use the array's name as a device address, so
 // the first call on each device (with that device current) looks the address up
 // with cudaGetSymbolAddress and caches it; that first call should come before any
-// stream capture.  All calls share the one array and it keeps the last call's
-// contents, so calls that overlap on the GPU (on different streams, or from
-// different host threads) race on it and must be serialised by the caller.  The
+// stream capture.  The address is kept for the life of the process: after a
+// cudaDeviceReset on a device the entry point must not be used there again.  All
+// calls share the one array and it keeps the last call's contents, so calls
+// issued in order on one stream are safe, while calls that can overlap on the
+// GPU (on different streams, or from different host threads) race on it and
+// must be serialised by the caller.  The
 // status word is cleared at the start of every call; the chunk sums are fully
 // written before they are read.
 #include <mutex>

@@ -4,6 +4,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "semicrf_internal.h"
 
 namespace semicrf {
@@ -23,6 +25,25 @@ int round_up_pow2(int v, int lo)
     return x;
 }
 }  // namespace
+
+int device_sm_count()
+{
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return 148;
+    }
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
 
 void prof_reset() { g_prof_i = 0; }
 
@@ -472,6 +493,7 @@ GoldArgs gold_args(const semicrf_dims *dims, const Layout &lay, void *ws, const 
     g.cntD = at<int32_t>(ws, lay.gcD);
     g.cntN = at<int32_t>(ws, lay.gcN);
     g.status = at<int32_t>(ws, lay.status);
+    g.wsign = 1.0;
     return g;
 }
 }  // namespace
@@ -512,6 +534,55 @@ semicrf_status semicrf_gold_backward(const semicrf_dims *dims, const int32_t *le
     int n = 0;
     cudaError_t e = launch_gold_backward(g, static_cast<cudaStream_t>(stream), &n);
     return finish(e, n);
+}
+
+semicrf_status semicrf_nll(const semicrf_dims *dims, const double *S, const float *A, const float *D,
+                           const int32_t *lengths, const int32_t *labels, const uint8_t *seg_start, double *logZ,
+                           double *score, double *nll, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!nll || !score || !logZ) return SEMICRF_ERR_INVALID_ARG;
+    semicrf_status s = semicrf_forward(dims, S, A, D, lengths, logZ, ws, ws_bytes, stream);
+    if (s != SEMICRF_OK) return s;
+    const int nf = g_last_launches;
+    Plan p;
+    Layout lay;
+    s = prepare(dims, SEMICRF_WS_TRAIN, ws, ws_bytes, &p, &lay);
+    if (s != SEMICRF_OK) return s;
+    if (!labels || !seg_start) return SEMICRF_ERR_INVALID_ARG;
+    GoldArgs g = gold_args(dims, lay, ws, lengths, labels, seg_start);
+    g.S = S;
+    g.A = A;
+    g.D = D;
+    g.score = score;
+    g.logZ = logZ;
+    g.nll = nll;
+    int n = 0;
+    cudaError_t e = launch_gold_score(g, static_cast<cudaStream_t>(stream), &n);
+    return finish(e, nf + n);
+}
+
+semicrf_status semicrf_nll_backward(const semicrf_dims *dims, const double *S, const float *A, const float *D,
+                                    const int32_t *lengths, const int32_t *labels, const uint8_t *seg_start,
+                                    const double *grad_nll, void *ws, size_t ws_bytes, float *dX, double *dA,
+                                    double *dD, void *stream)
+{
+    if (!labels || !seg_start) return SEMICRF_ERR_INVALID_ARG;
+    semicrf_status s = semicrf_backward(dims, S, A, D, lengths, grad_nll, ws, ws_bytes, dX, dA, dD, stream);
+    if (s != SEMICRF_OK) return s;
+    const int nb = g_last_launches;
+    Plan p;
+    Layout lay;
+    s = prepare(dims, SEMICRF_WS_TRAIN, ws, ws_bytes, &p, &lay);
+    if (s != SEMICRF_OK) return s;
+    GoldArgs g = gold_args(dims, lay, ws, lengths, labels, seg_start);
+    g.grad = grad_nll;
+    g.wsign = -1.0;   // the NLL subtracts the gold score
+    g.dX = dX;
+    g.dA = dA;
+    g.dD = dD;
+    int n = 0;
+    cudaError_t e = launch_gold_backward(g, static_cast<cudaStream_t>(stream), &n);
+    return finish(e, nb + n);
 }
 
 semicrf_status semicrf_viterbi(const semicrf_dims *dims, const double *S, const float *A, const float *D,
@@ -574,6 +645,25 @@ const char *semicrf_status_string(semicrf_status s)
     case SEMICRF_ERR_INVALID_SEGMENTATION: return "malformed gold segmentation";
     }
     return "unknown status";
+}
+
+semicrf_status semicrf_chain_plan(const semicrf_dims *dims, int32_t path, int32_t *info, int32_t n)
+{
+    semicrf_status s = check_dims_impl(dims);
+    if (s != SEMICRF_OK) return s;
+    if (!info || n < 9 || path < 0 || path > 2) return SEMICRF_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) info[i] = 0;
+    if (small_path_ok(dims->K, dims->C)) {
+        info[0] = 0;   // one CTA per sequence (warp-specialised team kernels)
+        info[1] = 1;
+        info[8] = path == 0 ? 2 * dims->B : dims->B;
+        info[7] = -1;
+        return SEMICRF_OK;
+    }
+    info[0] = 1;
+    if (!cl_plan_info(dims->K, dims->C, path, info + 1)) return SEMICRF_ERR_UNSUPPORTED_SHAPE;
+    info[8] = path == 0 ? 2 * dims->B : dims->B;
+    return SEMICRF_OK;
 }
 
 int32_t semicrf_last_launch_count(void) { return g_last_launches; }

@@ -85,6 +85,10 @@ struct Layout {
     size_t total = 0;
 };
 
+// Streaming multiprocessors of the current device (cached per device; 148, the
+// B200 count, when no device can be queried, e.g. on a host without a GPU).
+int device_sm_count();
+
 // Optional per-launch event recording (semicrf_set_profile_events).
 void prof_before(cudaStream_t st);
 void prof_after(cudaStream_t st);
@@ -147,6 +151,9 @@ cudaError_t launch_cl_forward(const FbArgs &a, cudaStream_t st, bool recompute);
 cudaError_t launch_cl_backward(const FbArgs &a, cudaStream_t st);
 // Forward storing its rows and the beta chain in one launch (2B clusters).
 cudaError_t launch_cl_fused(const FbArgs &a, cudaStream_t st);
+// Planner's choice for path 0 (fused), 1 (forward) or 2 (backward) and how many
+// such clusters the GPU holds at once (see semicrf_chain_plan).
+bool cl_plan_info(int K, int C, int path, int32_t *info);
 // dD and dA from the cluster backward's stored rows (cl_grads.cu): two contraction
 // kernels writing split partial sums, one kernel reducing them (3 launches).
 constexpr int kGradChunk = 64;   // start positions per staged chunk
@@ -208,7 +215,10 @@ struct GoldArgs {
     const int32_t *lengths, *labels;
     const uint8_t *seg_start;
     const double *grad;   // backward weights, NULL: ones
+    double wsign;         // the weights are wsign * grad[b] (wsign * 1 when grad is NULL)
     double *score;
+    const double *logZ;   // when set with nll: nll[b] = logZ[b] - score[b]
+    double *nll;
     float *dX;
     double *dA, *dD;
     int32_t *cntA, *cntD, *cntN;

@@ -410,7 +410,8 @@ __global__ void __launch_bounds__(256) team_finalise_kernel(FbArgs a, int ppb)
 int team_post_splits(int B, int T)
 {
     const long long Q = (long long)B * ((T + kPC - 1) / kPC);
-    return (int)(Q < 2 * 148 ? Q : 2 * 148);
+    const int cap = 2 * device_sm_count();
+    return (int)(Q < cap ? Q : cap);
 }
 
 int team_post_chunks(int T) { return (T + kPC - 1) / kPC; }
@@ -428,7 +429,8 @@ cudaError_t launch_team_post(const FbArgs &a, cudaStream_t st)
     if (ppb < 1) ppb = 1;
     const int nP = (int)(((long long)(a.C * a.C + a.K * a.C) * 32 + 255) / 256);
     prof_before(st);
-    team_finalise_kernel<<<(unsigned)(a.B * ppb + (nP < 148 ? nP : 148)), 256, 0, st>>>(a, (int)ppb);
+    const int nsm = device_sm_count();
+    team_finalise_kernel<<<(unsigned)(a.B * ppb + (nP < nsm ? nP : nsm)), 256, 0, st>>>(a, (int)ppb);
     prof_after(st);
     return cudaGetLastError();
 }

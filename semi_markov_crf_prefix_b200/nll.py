@@ -3,16 +3,19 @@ log Z_b - score_b(y*) (Streaming Structured Inference with Flash-SemiCRF,
 technical summary section 3), as a torch.autograd.Function over the library's
 kernels.
 
-Forward: prefix scan, streaming forward (log Z) and the gold-score kernel.
-Backward: the library's backward with weights g (gradient of g . log Z) and the
-gold backward with weights -g (adds the gradient of -g . score).  Argument
-marshalling only; every step runs in libsemicrf.so.
+Forward: semicrf_nll -- prefix scan, streaming forward with checkpoints (log Z),
+the gold-score kernel and nll = log Z - score, all on the device.
+Backward: semicrf_nll_backward -- the checkpointed backward with the upstream
+weights g and the gold-segmentation counts with weights -g.  Argument
+marshalling only; every step runs in libsemicrf.so.  The checkpointed pair is
+used (not the side-by-side step) because the upstream weights are known only
+when the backward runs, and the pair keeps O(sqrt(T) K C) state between the two.
 """
 from __future__ import annotations
 
 import torch
 
-from . import backward, forward, gold_backward, gold_score, new_workspace, prefix_scan, WS_TRAIN
+from . import WS_TRAIN, new_workspace, nll, nll_backward, prefix_scan
 
 
 class SemiCRFNLL(torch.autograd.Function):
@@ -25,18 +28,17 @@ class SemiCRFNLL(torch.autograd.Function):
         Dc = D.detach().contiguous().float()
         ws = new_workspace(B, T, K, C, WS_TRAIN, ckpt_interval, device=x.device)
         S, _ = prefix_scan(xc, lengths, ws=ws)
-        logZ, ws = forward(S, Ac, Dc, lengths, ws=ws, ckpt_interval=ckpt_interval)
-        score = gold_score(S, Ac, Dc, lengths, labels, seg_start, ws)
+        out, _, _ = nll(S, Ac, Dc, lengths, labels, seg_start, ws, ckpt_interval=ckpt_interval)
         ctx.save_for_backward(S, Ac, Dc, lengths, labels, seg_start, ws)
         ctx.ckpt_interval = ckpt_interval
         ctx.dtypes = (x.dtype, A.dtype, D.dtype)
-        return logZ - score
+        return out
 
     @staticmethod
     def backward(ctx, g):
         S, Ac, Dc, lengths, labels, seg_start, ws = ctx.saved_tensors
         g = g.detach().to(torch.float64).contiguous()
-        dX, dA, dD = backward(S, Ac, Dc, lengths, ws, grad_logZ=g, ckpt_interval=ctx.ckpt_interval)
-        gold_backward(lengths, labels, seg_start, ws, dX, dA, dD, grad_score=(-g).contiguous())
+        dX, dA, dD = nll_backward(S, Ac, Dc, lengths, labels, seg_start, ws, grad_nll=g,
+                                  ckpt_interval=ctx.ckpt_interval)
         tx, tA, tD = ctx.dtypes
         return dX.to(tx), dA.to(tA), dD.to(tD), None, None, None, None

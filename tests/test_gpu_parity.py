@@ -96,7 +96,7 @@ def check_against_oracle(w, g, grad=None, precision=True):
     return o
 
 
-def check_viterbi(w, g):
+def check_viterbi(w, g, ref=None):
     """Viterbi against the oracle.  The best score is unique, and so are the
     per-position labels on continuous inputs.  The segment starts are not: two
     adjacent segments of one label with durations d and d' score exactly the same
@@ -106,8 +106,9 @@ def check_viterbi(w, g):
     pick which side wins.  So: score and labels as the oracle's; segment starts
     equal to the oracle's or, for a sequence where they differ, a valid
     segmentation whose score, recomputed by the oracle from the definition, is
-    the optimum to rounding."""
-    s, labels, seg = oracle.viterbi(w.x, w.A, w.D, w.lengths)
+    the optimum to rounding.  ref: the oracle's (score, labels, seg_start) when
+    already computed."""
+    s, labels, seg = oracle.viterbi(w.x, w.A, w.D, w.lengths) if ref is None else ref
     np.testing.assert_allclose(g["score"], s, rtol=1e-12)
     assert np.array_equal(g["labels"], labels)
     differ = [b for b in range(w.B) if not np.array_equal(g["seg_start"][b], seg[b])]

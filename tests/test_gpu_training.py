@@ -158,3 +158,32 @@ def test_gold_malformed_segmentation_reports_status():
         S, _ = sc.prefix_scan(x, lens, ws=ws)
         sc.gold_score(S, A, D, lens, torch.from_numpy(lb).to(dev), torch.from_numpy(sg).to(dev), ws)
         assert sc.device_status(ws) == sc._lib.SEMICRF_ERR_INVALID_SEGMENTATION
+
+
+def test_nll_entry_points():
+    # semicrf_nll forms log Z - score on the device from the same log Z and score
+    # the separate calls give; semicrf_nll_backward equals the backward with
+    # weights g followed by the gold backward with weights -g
+    import torch
+    import semi_markov_crf_prefix_b200 as sc
+    w = wl.make_workload("ner", B=6)
+    labels, seg = _random_segmentations(w, seed=5)
+    dev, x, A, D, lens = _dev(w)
+    lb, sg = torch.from_numpy(labels).to(dev), torch.from_numpy(seg).to(dev)
+    g = torch.linspace(-1.0, 2.0, w.B, dtype=torch.float64, device=dev)
+    ws = sc.new_workspace(w.B, w.T, w.K, w.C, sc.WS_TRAIN, device=dev)
+    sc.clear_device_status(ws)
+    S, _ = sc.prefix_scan(x, lens, ws=ws)
+    nll, logZ, score = sc.nll(S, A, D, lens, lb, sg, ws)
+    dX, dA, dD = sc.nll_backward(S, A, D, lens, lb, sg, ws, grad_nll=g)
+    assert sc.device_status(ws) == 0
+    ws2 = sc.new_workspace(w.B, w.T, w.K, w.C, sc.WS_TRAIN, device=dev)
+    logZ2, _ = sc.forward(S, A, D, lens, ws=ws2)
+    score2 = sc.gold_score(S, A, D, lens, lb, sg, ws2)
+    rX, rA, rD = sc.backward(S, A, D, lens, ws2, grad_logZ=g)
+    sc.gold_backward(lens, lb, sg, ws2, rX, rA, rD, grad_score=(-g).contiguous())
+    assert sc.device_status(ws2) == 0
+    assert torch.equal(logZ, logZ2) and torch.equal(score, score2)
+    assert torch.equal(nll, logZ2 - score2)
+    for a, b in ((dX, rX), (dA, rA), (dD, rD)):
+        assert torch.equal(a, b)
