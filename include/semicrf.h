@@ -282,7 +282,10 @@ const char *semicrf_status_string(semicrf_status s);
  * Launch geometry of the sequential chains for these dims, for tuning and
  * diagnostics (no counterpart on the pages).  path: 0 the forward_backward
  * step (forward and backward chains in one launch), 1 semicrf_forward,
- * 2 semicrf_backward.  Fills info[0..8] (n >= 9):
+ * 2 semicrf_backward.  The geometry is the one the launch uses: the cheapest by
+ * the library's cost model among those of which the current device holds all
+ * of the launch's clusters at once (the cheapest overall if none does).
+ * Fills info[0..8] (n >= 9):
  *   info[0]  kernel family: 0 = one CTA per sequence (C <= 32 and K <= 32),
  *            1 = one thread-block cluster per chain
  *   info[1]  CTAs per cluster G      info[2] threads per CTA

@@ -414,7 +414,7 @@ def nll_backward(S, A, D, lengths, labels, seg_start, ws, grad_nll=None, ckpt_in
 def semicrf_nll(x, A, D, lengths, labels, seg_start, ckpt_interval=0):
     """Negative log-likelihood log Z_b - score_b(gold) [B] float64, differentiable
     with respect to x, A and D (torch.autograd)."""
-    from .nll import SemiCRFNLL
+    from .training import SemiCRFNLL
     return SemiCRFNLL.apply(x, A, D, lengths, labels, seg_start, ckpt_interval)
 
 

@@ -59,12 +59,25 @@ def _compile(src: Path, verbose: bool) -> Path:
     return obj
 
 
+def _stale(src: Path, force: bool) -> bool:
+    """An object needs compiling when it is missing or older than its source or any header."""
+    obj = BUILD / (src.stem + ".o")
+    if force or not obj.exists():
+        return True
+    t = obj.stat().st_mtime
+    headers = list(CSRC.glob("*.h")) + list(CSRC.glob("*.cuh")) + list(INCLUDE.glob("*.h"))
+    return any(p.stat().st_mtime > t for p in [src, *headers])
+
+
 def build(force: bool = False, verbose: bool = False) -> Path:
     if not force and up_to_date():
         return LIB
     BUILD.mkdir(exist_ok=True)
+    srcs = sources()
+    todo = [s for s in srcs if _stale(s, force or verbose)]
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), sources()))
+        list(ex.map(lambda s: _compile(s, verbose), todo))
+    objs = [BUILD / (s.stem + ".o") for s in srcs]
     tmp = LIB.with_suffix(".so.tmp")
     cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", str(tmp), *map(str, objs)]
     r = subprocess.run(cmd, capture_output=True, text=True)

@@ -45,6 +45,13 @@
 #include <stdio.h>
 #include <stdlib.h>
 
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <utility>
+#include <vector>
+
 #include "device_util.cuh"
 #include "semicrf_internal.h"
 
@@ -124,22 +131,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
     }
 }
 
-// Store v at the address of `local` in CTA `rank` of the cluster and complete 8
-// bytes on that CTA's copy of `bar`.
-__device__ __forceinline__ void st_async_f64(const double *local, const uint64_t *bar, uint32_t rank, double v)
+// st.async of v to the shared::cluster address ra, completing 8 bytes on the
+// mbarrier at the shared::cluster address rb (both from mapa, done once).
+__device__ __forceinline__ void st_async_at(uint32_t ra, uint32_t rb, double v)
 {
-    uint32_t ra, rb;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_addr(local)), "r"(rank));
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(smem_addr(bar)), "r"(rank));
     asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];" ::"r"(ra),
                  "l"(__double_as_longlong(v)), "r"(rb)
                  : "memory");
 }
 
-// xor-shuffle sum over groups of `width` consecutive lanes (width a power of two <= 32)
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t local, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+
+// xor-shuffle sum over groups of `width` consecutive lanes (width a power of two
+// <= 32): offsets width/2, ..., 1 in that order, unrolled
 __device__ __forceinline__ double group_sum(double v, int width)
 {
-    for (int off = width >> 1; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        if (off < width) v += __shfl_xor_sync(0xffffffffu, v, off);
     return v;
 }
 
@@ -148,9 +162,9 @@ __device__ __forceinline__ double rescale(double x, int h) { return h == 0 ? x :
 
 // Shared memory of both chains (the backward uses the pf_cu/pf_ca/pf_eu/pf_ea rings).
 struct ClSmem {
-    double *ring;    // [2K][RS] every row twice
-    double *Wd;      // [K][RS]  exp(D)
-    double *gath;    // [2][C]   a' (forward) or bp (backward) of the position, all labels
+    double *ring;    // [2K][RS] every row twice, with LPW zero rows before and after
+    double *Wd;      // [K][RS]  exp(D), when the window lanes do not hold it in registers
+    double *gath;    // [2][GP]  a' (forward) or bp (backward) of the position, all labels (zeros past C)
     double *qbuf;    // [Cg]     transition result of each label, for its owner
     double *pre3;    // [4][Cg][PW] window sums two positions ahead
     double *pf_es, *pf_ies, *pf_cu, *pf_ca;   // [kPF][Cg] prefetch rings
@@ -158,23 +172,25 @@ struct ClSmem {
     int *pf_m, *pf_eu, *pf_ea;                // [kPF][Cg] each
     int *hbuf;       // [2][Cg] rebase exponent of each label at the last two positions
     int *kbuf;       // [4]     normaliser exponents
+    uint32_t *rmap;  // [32*NWO][16] mapped destination of each owner lane's value, per CTA of the cluster
 };
 
 __host__ __device__ __forceinline__ size_t cl_smem_bytes_impl(int K, int C, const ClGeom &g, bool bwd)
 {
     const size_t npf = bwd ? 4 : 2;
-    const size_t nd = 3 * (size_t)K * g.RS + 2 * (size_t)C + g.Cg + 4 * (size_t)g.Cg * g.PW + npf * kPF * g.Cg;
-    const size_t ni = (bwd ? 3 : 1) * (size_t)kPF * g.Cg + 2 * (size_t)g.Cg + 4;
+    const size_t nd = ((g.NRB > 0 ? 2 : 3) * (size_t)K + 2 * (size_t)g.PAD) * g.RS + 2 * (size_t)g.GP + g.Cg +
+                      4 * (size_t)g.Cg * g.PW + npf * kPF * g.Cg;
+    const size_t ni = (bwd ? 3 : 1) * (size_t)kPF * g.Cg + 2 * (size_t)g.Cg + 4 + 32 * 16 * (size_t)g.NWO;
     return nd * sizeof(double) + 2 * sizeof(uint64_t) + ni * sizeof(int);
 }
 
 __device__ __forceinline__ ClSmem cl_smem(double *base, int K, int C, const ClGeom &g, bool bwd)
 {
     ClSmem s;
-    s.ring = base;
-    s.Wd = s.ring + 2 * (size_t)K * g.RS;
-    s.gath = s.Wd + (size_t)K * g.RS;
-    s.qbuf = s.gath + 2 * C;
+    s.ring = base + (size_t)g.PAD * g.RS;
+    s.Wd = s.ring + (2 * (size_t)K + g.PAD) * g.RS;
+    s.gath = s.Wd + (g.NRB > 0 ? 0 : (size_t)K * g.RS);
+    s.qbuf = s.gath + 2 * (size_t)g.GP;
     s.pre3 = s.qbuf + g.Cg;
     s.pf_es = s.pre3 + 4 * g.Cg * g.PW;
     s.pf_ies = s.pf_es + kPF * g.Cg;
@@ -187,6 +203,7 @@ __device__ __forceinline__ ClSmem cl_smem(double *base, int K, int C, const ClGe
     s.pf_ea = bwd ? s.pf_eu + kPF * g.Cg : s.pf_eu;
     s.hbuf = bwd ? s.pf_ea + kPF * g.Cg : s.pf_eu;
     s.kbuf = s.hbuf + 2 * g.Cg;
+    s.rmap = reinterpret_cast<uint32_t *>(s.kbuf + 4);
     return s;
 }
 
@@ -277,21 +294,125 @@ __device__ __forceinline__ double window_bwd(double *ring, const double *Wd, int
     return strided_dot(ring + (size_t)(sK + i0) * RS + lc, step, Wd + (size_t)(i0 + 1) * RS + lc, step, n);
 }
 
-// Normaliser sum n = sum_c g[c] over one warp: C/32 loads per lane, a tree, five
-// shuffle levels.  Every lane gets n; every CTA forms it in the same order.
-__device__ __forceinline__ double warp_total(const double *g, int C, int lane)
+// The same window sums with the lane's weights in registers (W[m] for row m of
+// the lane, 0 past the last duration) and no per-row bounds: NR rows per lane
+// (a bucket >= the rows the lane has), the rows beyond the window read the
+// ring's zero padding or older finite rows, times weight 0.  Four interleaved
+// partial sums.
+template <int NR, int NU>
+__device__ __forceinline__ double window_fwd_reg(double *ring, int K, int RS, int lc, int LPW, int j, int tauK,
+                                                 int hp, const double (&W)[NU])
 {
-    double acc = 0.0;
-    for (int i0 = 0; i0 < C; i0 += 128) {
-        double v[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int i = i0 + 32 * k + lane;
-            v[k] = i < C ? g[i] : 0.0;
+    static_assert(NR <= NU, "window rows exceed the register array");
+    const int d0 = 3 + j;
+    if (hp != 0 && d0 <= K) {
+        const int n = (K - d0) / LPW + 1;
+        for (int m = 0; m < n; ++m) {
+            const int d = d0 + m * LPW;
+            if (d < 4) continue;
+            const int sl = tauK + K - d;
+            const int other = sl >= K ? sl - K : sl + K;
+            const double v = rescale(ring[sl * RS + lc], hp);
+            ring[sl * RS + lc] = v;
+            ring[other * RS + lc] = v;
         }
-        acc += (v[0] + v[1]) + (v[2] + v[3]);
     }
-    return group_sum(acc, 32);
+    const double *p = ring + (tauK + K - d0) * RS + lc;
+    const int step = LPW * RS;
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+    for (int m = 0; m < NR; ++m) acc[m & 3] = fma(p[-m * step], W[m], acc[m & 3]);
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+template <int NR, int NU>
+__device__ __forceinline__ double window_bwd_reg(double *ring, int K, int RS, int lc, int LPW, int j, int sK, int hp,
+                                                 const double (&W)[NU])
+{
+    static_assert(NR <= NU, "window rows exceed the register array");
+    const int i0 = 1 + j;
+    if (hp != 0 && i0 <= K - 2) {
+        const int n = (K - 2 - i0) / LPW + 1;
+        for (int m = 0; m < n; ++m) {
+            const int i = i0 + m * LPW;
+            if (i < 2) continue;
+            const int sl = sK + i;
+            const int other = sl >= K ? sl - K : sl + K;
+            const double v = rescale(ring[sl * RS + lc], hp);
+            ring[sl * RS + lc] = v;
+            ring[other * RS + lc] = v;
+        }
+    }
+    const double *p = ring + (sK + i0) * RS + lc;
+    const int step = LPW * RS;
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+    for (int m = 0; m < NR; ++m) acc[m & 3] = fma(p[m * step], W[m], acc[m & 3]);
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// Window sum with the row count of the plan's bucket (8, 16 or 32 rows per lane).
+template <int NU>
+__device__ __forceinline__ double window_fwd_nr(int NRB, double *ring, int K, int RS, int lc, int LPW, int j,
+                                                int tauK, int hp, const double (&W)[NU])
+{
+    if constexpr (NU >= 32)
+        if (NRB == 32) return window_fwd_reg<32, NU>(ring, K, RS, lc, LPW, j, tauK, hp, W);
+    if (NRB == 16) return window_fwd_reg<16, NU>(ring, K, RS, lc, LPW, j, tauK, hp, W);
+    return window_fwd_reg<8, NU>(ring, K, RS, lc, LPW, j, tauK, hp, W);
+}
+
+template <int NU>
+__device__ __forceinline__ double window_bwd_nr(int NRB, double *ring, int K, int RS, int lc, int LPW, int j, int sK,
+                                                int hp, const double (&W)[NU])
+{
+    if constexpr (NU >= 32)
+        if (NRB == 32) return window_bwd_reg<32, NU>(ring, K, RS, lc, LPW, j, sK, hp, W);
+    if (NRB == 16) return window_bwd_reg<16, NU>(ring, K, RS, lc, LPW, j, sK, hp, W);
+    return window_bwd_reg<8, NU>(ring, K, RS, lc, LPW, j, sK, hp, W);
+}
+
+// Pairwise sum of N values (N a power of two).
+template <int N>
+__device__ __forceinline__ double tree_sum(const double (&x)[N])
+{
+    double p[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) p[i] = x[i];
+#pragma unroll
+    for (int w = N; w > 1; w >>= 1) {
+#pragma unroll
+        for (int i = 0; i < w / 2; ++i) p[i] = p[2 * i] + p[2 * i + 1];
+    }
+    return p[0];
+}
+
+// sum_m v[m] E[m] with v[m] = gp[m * stride], and the plain sum of the v[m]
+// into *vsum: chunks of eight (loads, a product tree, a sum tree) combined
+// pairwise, so that at most a chunk of loaded values is live.
+template <int N>
+__device__ __forceinline__ double chunked_dot(const double *gp, int stride, const double (&E)[N], double *vsum)
+{
+    if constexpr (N <= 8) {
+        double v[N];
+#pragma unroll
+        for (int m = 0; m < N; ++m) v[m] = gp[m * stride];
+        *vsum = tree_sum<N>(v);
+        return tree_dot<N>(v, E);
+    } else {
+        double part[N / 8], sums[N / 8];
+#pragma unroll
+        for (int c8 = 0; c8 < N / 8; ++c8) {
+            double v[8];
+            const double(&e8)[8] = *reinterpret_cast<const double(*)[8]>(&E[c8 * 8]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = gp[(c8 * 8 + i) * stride];
+            part[c8] = tree_dot<8>(v, e8);
+            sums[c8] = tree_sum<8>(v);
+        }
+        *vsum = tree_sum<N / 8>(sums);
+        return tree_sum<N / 8>(part);
+    }
 }
 
 // Roles of a thread: owner warps (label lc = lane of the warp's 32), then
@@ -353,7 +474,6 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
     extern __shared__ __align__(16) double smc[];
     const int K = a.K, C = a.C, Cg = g.Cg, NT = g.NT, RS = g.RS, PW = g.PW;
     const int NOT = 32 * (g.NWO + g.NWT);   // owner + transition threads
-    const int NXW = 32 * (1 + g.NWT);       // owner warp 0 + transition threads
     const int W0T = 32 * (g.NWO + g.NWT);   // first window thread
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rank = CLUSTER ? (int)cluster_rank() : 0;
@@ -395,7 +515,7 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
         for (int i = tid; i < K * Cg; i += NT) {
             const int sl = i / Cg, l2 = i % Cg;
             const bool ok = l2 < cg_own;
-            sm.Wd[sl * RS + l2] = ok ? exp((double)a.D[(size_t)sl * C + c0l + l2]) : 0.0;
+            if (g.NRB == 0) sm.Wd[sl * RS + l2] = ok ? exp((double)a.D[(size_t)sl * C + c0l + l2]) : 0.0;
             double v;
             if constexpr (RECOMPUTE) {
                 v = ok ? ck_ring[(size_t)sl * C + c0l + l2] : 0.0;
@@ -406,7 +526,11 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
             sm.ring[sl * RS + l2] = v;
             sm.ring[(sl + K) * RS + l2] = v;
         }
-        for (int i = tid; i < 2 * C; i += NT) sm.gath[i] = 0.0;
+        for (int i = tid; i < g.PAD * RS; i += NT) {   // the zero rows around the ring
+            sm.ring[i - g.PAD * RS] = 0.0;
+            sm.ring[2 * K * RS + i] = 0.0;
+        }
+        for (int i = tid; i < 2 * g.GP; i += NT) sm.gath[i] = 0.0;
         for (int i = tid; i < 4 * Cg * PW; i += NT) sm.pre3[i] = 0.0;
         for (int i = tid; i < 2 * Cg; i += NT) sm.hbuf[i] = 0;
         if (tid == 0) {
@@ -435,29 +559,56 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
         }
     }
     __syncthreads();
-    // window sums for the first two positions, from the restored ring (one reference)
-    if (ro.is_win) {
-        for (int q = 1; q <= 2; ++q) {
-            const int tau = t0 + q;
-            const double v = ro.lab_ok ? window_fwd(sm.ring, sm.Wd, K, RS, lc, g.LPW, j, tau % K, 0) : 0.0;
-            const double s = group_sum(v, g.LPW < 32 ? g.LPW : 32);
-            if (ro.lab_ok && (j & 31) == 0) sm.pre3[(q - 1) * Cg * PW + lc * PW + (j >> 5)] = s;
-        }
-    }
-    // One register array holds either the transition weights E (transition lanes)
-    // or the chain state (owner lanes): a thread has one role, and sharing keeps
-    // the register count of the kernel that of the larger of the two.
+    // One register array holds the transition weights E (transition lanes), the
+    // window weights exp(D) of the lane's rows (window lanes, when they fit) or
+    // the chain state (owner lanes): a thread has one role, and sharing keeps
+    // the register count of the kernel that of the largest of the three.
     // Chain state at the start of step t: U1 = U[t-1], U2 = U[t-2] (reference of
     // t-1) and the values prepared for t from everything but U[t-1]:
     //   pre = U[t-2] W1 + pre3_t,  e = exp(S_t + ln2 (r - k_t)),  f = exp(ln2 (k_t - r) - S_t),
     //   pe = pre e,  w0e = W0 e,  so a'[t] = U[t-1] w0e + pe is one FMA after U[t-1].
-    constexpr int NU = CPL > 10 ? CPL : 10;
+    constexpr int NU = CPL > 16 ? CPL : 16;
+    const int nrw = K > 2 ? (K - 2 + g.LPW - 1) / g.LPW : 0;   // window rows per lane
+    const bool wreg = g.NRB > 0;
     double R[NU];
 #pragma unroll
     for (int m = 0; m < NU; ++m) {
         const int cp = j + m * g.LPL;
-        R[m] = (m < CPL && ro.is_tr && ro.lab_ok && cp < C) ? exp((double)a.A[(size_t)cp * C + c]) : 0.0;
+        double v = 0.0;
+        if (m < CPL && ro.is_tr && ro.lab_ok && cp < C) v = exp((double)a.A[(size_t)cp * C + c]);
+        const int d = 3 + j + m * g.LPW;   // window lanes: duration of row m
+        if (ro.is_win && wreg && ro.lab_ok && m < nrw && d <= K) v = exp((double)a.D[(size_t)(d - 1) * C + c]);
+        R[m] = v;
     }
+    // window sums for the first two positions, from the restored ring (one reference)
+    if (ro.is_win) {
+        for (int q = 1; q <= 2; ++q) {
+            const int tau = t0 + q;
+            double v = 0.0;
+            if (ro.lab_ok)
+                v = wreg ? window_fwd_nr<NU>(g.NRB, sm.ring, K, RS, lc, g.LPW, j, tau % K, 0, R)
+                         : window_fwd(sm.ring, sm.Wd, K, RS, lc, g.LPW, j, tau % K, 0);
+            const double s = group_sum(v, g.LPW < 32 ? g.LPW : 32);
+            if (ro.lab_ok && (j & 31) == 0) sm.pre3[(q - 1) * Cg * PW + lc * PW + (j >> 5)] = s;
+        }
+    }
+    // The exchange: each owner label's value goes to every CTA of the cluster.
+    // With one owner warp and at most 16 labels per CTA the warp's upper half
+    // sends the upper half of the ranks (the value shuffled from the lower half).
+    // Destination addresses are mapped once.
+    const bool split = CLUSTER && g.NWO == 1 && Cg <= 16 && g.G >= 2;
+    const int slab = split ? (lane & 15) : lc;
+    const bool sends = ro.is_own && slab < cg_own && (split || ro.lab_ok);
+    const int gcnt = split ? g.G / 2 : g.G;
+    // each owner lane's destinations are mapped once into shared memory; a CTA's
+    // shared window maps contiguously, so the mbarrier's mapped address is the
+    // value slot's plus the same offset as locally
+    const uint32_t gloc = smem_addr(&sm.gath[c0l + slab]);
+    uint32_t *rmap = sm.rmap + (size_t)(ro.is_own ? tid : 0) * 16;   // owner threads are 0 .. 32 NWO - 1
+    if (CLUSTER && sends)
+        for (int k = 0; k < gcnt; ++k)
+            rmap[k] = mapa_rank(gloc, (uint32_t)((split && lane >= 16 ? g.G / 2 : 0) + k));
+    const uint32_t bar_off = smem_addr(&sm.full[0]) - gloc;
     double(&E)[CPL] = *reinterpret_cast<double(*)[CPL]>(&R[0]);
     double &W0 = R[0], &W1 = R[1], &U1 = R[2], &U2 = R[3], &pre = R[4], &f = R[5], &pe = R[6], &w0e = R[7],
            &ap = R[8];
@@ -489,8 +640,8 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
         w0e_o = W0 * e;
     };
     if (own) {
-        W0 = sm.Wd[lc];
-        W1 = K >= 2 ? sm.Wd[RS + lc] : 0.0;
+        W0 = exp((double)a.D[c]);
+        W1 = K >= 2 ? exp((double)a.D[C + c]) : 0.0;
         U1 = sm.ring[(t0 % K) * RS + lc];
         U2 = K >= 2 ? sm.ring[(((t0 - 1) % K + K) % K) * RS + lc] : 0.0;
         if constexpr (RECOMPUTE) {
@@ -516,13 +667,21 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
         const int par = u & 1;
         if (ro.is_own) {
             // ------------------------------------------------ owners: chain
-            if (own) {
-                ap = fma(U1, w0e, pe);
-                if constexpr (CLUSTER) {
-                    for (int g2 = 0; g2 < g.G; ++g2) st_async_f64(&sm.gath[par * C + c], &sm.full[par], g2, ap);
-                } else {
-                    sm.gath[par * C + c] = ap;
+            if (own) ap = fma(U1, w0e, pe);
+            if constexpr (CLUSTER) {
+                const double sv = split ? __shfl_sync(0xffffffffu, ap, lane & 15) : ap;
+                if (sends) {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        if (k < gcnt) {
+                            const uint32_t ra = rmap[k];
+                            st_async_at(ra + par * g.GP * 8, ra + bar_off + par * 8, sv);
+                        }
                 }
+            } else if (own) {
+                sm.gath[par * g.GP + c] = ap;
+            }
+            if (own) {
                 // rebase when p = a' / e leaves [2^-512, 2^512]
                 const double p = fma(U1, W0, pre);
                 const int ex = exponent_of(p);
@@ -545,29 +704,6 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
                 cta_arrive(1, NOT);   // a'[t] stored (for the transition warps)
                 if (g.NWO > 1) cta_barrier(7, 32 * g.NWO);
                 else __syncwarp();
-            }
-            if (warp == 0) {
-                // normaliser n_t = sum_c a'[t,c] (the same in every CTA)
-                if (!wait_values<CLUSTER>(sm, par, u, timed_out)) {
-                    timed_out = true;
-                    set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
-                }
-                if constexpr (CLUSTER) cta_arrive(5, NXW);   // a'[t] of every label has arrived
-                const double n = warp_total(sm.gath + par * C, C, lane);
-                if (lane == 0) {
-                    const int kk = sm.kbuf[u & 3];
-                    if (t == L) {
-                        if (!RECOMPUTE && rank == 0) {
-                            const double lz = kLn2 * (double)kk + log(n);
-                            a.logZ[b] = lz;
-                            a.lz[b].logn = log(n);
-                            a.lz[b].k = kk;
-                            if (!isfinite(lz)) set_status(a.status, SEMICRF_ERR_DEVICE_RANGE);
-                        }
-                    } else {
-                        sm.kbuf[(u + 2) & 3] = kk + exponent_of(n);
-                    }
-                }
             }
             cta_barrier(4, NOT);   // q[t] ready
             // ------------------------------------------------ owners: new row
@@ -593,23 +729,45 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
             }
         } else if (ro.is_tr) {
             // -------------------------------------------------------- transition
-            if constexpr (CLUSTER) cta_barrier(5, NXW);
-            else cta_barrier(1, NOT);
-            double v[CPL];
-#pragma unroll
-            for (int m = 0; m < CPL; ++m) {
-                const int cp = j + m * g.LPL;
-                v[m] = cp < C ? sm.gath[par * C + cp] : 0.0;
+            if constexpr (CLUSTER) {
+                if (!wait_values<CLUSTER>(sm, par, u, timed_out)) {
+                    timed_out = true;
+                    set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
+                }
+            } else {
+                cta_barrier(1, NOT);
             }
-            const double q = group_sum(tree_dot<CPL>(v, E), g.LPL);
+            const double *gp = sm.gath + par * g.GP + j;   // zeros past C
+            double vs;
+            const double q = group_sum(chunked_dot<CPL>(gp, g.LPL, E, &vs), g.LPL);
             if (ro.lab_ok && j == 0) sm.qbuf[lc] = q;
+            // normaliser n_t = sum_c a'[t,c]: the lanes of the first label sum the values
+            // they loaded, in the same order in every CTA
+            const double n = group_sum(vs, g.LPL);
+            if (lc == 0 && j == 0) {
+                const int kk = sm.kbuf[u & 3];
+                if (t == L) {
+                    if (!RECOMPUTE && rank == 0) {
+                        const double lz = kLn2 * (double)kk + log(n);
+                        a.logZ[b] = lz;
+                        a.lz[b].logn = log(n);
+                        a.lz[b].k = kk;
+                        if (!isfinite(lz)) set_status(a.status, SEMICRF_ERR_DEVICE_RANGE);
+                    }
+                } else {
+                    sm.kbuf[(u + 2) & 3] = kk + exponent_of(n);
+                }
+            }
             cta_arrive(4, NOT);
         } else if (ro.is_win) {
             // ------------------------------------- window sums two positions ahead
             if (CLUSTER && tid == W0T) mbar_expect_tx(&sm.full[par], C * 8);
             const int hp = ro.lab_ok ? sm.hbuf[(par ^ 1) * Cg + lc] : 0;   // rebase at t-1
-            const int tau2K = (tK + 2) % K;
-            const double v = ro.lab_ok ? window_fwd(sm.ring, sm.Wd, K, RS, lc, g.LPW, j, tau2K, hp) : 0.0;
+            const int tau2K = tK + 2 >= K ? tK + 2 - K : tK + 2;   // K >= 3 whenever a row is read
+            double v = 0.0;
+            if (ro.lab_ok)
+                v = wreg ? window_fwd_nr<NU>(g.NRB, sm.ring, K, RS, lc, g.LPW, j, tau2K, hp, R)
+                         : window_fwd(sm.ring, sm.Wd, K, RS, lc, g.LPW, j, tau2K, hp);
             const double s = group_sum(v, g.LPW < 32 ? g.LPW : 32);
             if (ro.lab_ok && (j & 31) == 0) sm.pre3[((u + 2) & 3) * Cg * PW + lc * PW + (j >> 5)] = s;
         }
@@ -661,7 +819,6 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
     extern __shared__ __align__(16) double smc[];
     const int K = a.K, C = a.C, Cg = g.Cg, NT = g.NT, RS = g.RS, PW = g.PW;
     const int NOT = 32 * (g.NWO + g.NWT);
-    const int NXW = 32 * (1 + g.NWT);
     const int W0T = 32 * (g.NWO + g.NWT);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rank = CLUSTER ? (int)cluster_rank() : 0;
@@ -684,13 +841,17 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
     for (int i = tid; i < K * Cg; i += NT) {
         const int sl = i / Cg, l2 = i % Cg;
         const bool ok = l2 < cg_own;
-        sm.Wd[sl * RS + l2] = ok ? exp((double)a.D[(size_t)sl * C + c0l + l2]) : 0.0;
+        if (g.NRB == 0) sm.Wd[sl * RS + l2] = ok ? exp((double)a.D[(size_t)sl * C + c0l + l2]) : 0.0;
         const size_t ixL = (rowbase + L) * C + c0l + l2;
         const double v = (ok && sl == L % K) ? a.tES[ixL] : 0.0;
         sm.ring[sl * RS + l2] = v;
         sm.ring[(sl + K) * RS + l2] = v;
     }
-    for (int i = tid; i < 2 * C; i += NT) sm.gath[i] = 0.0;
+    for (int i = tid; i < g.PAD * RS; i += NT) {   // the zero rows around the ring
+        sm.ring[i - g.PAD * RS] = 0.0;
+        sm.ring[2 * K * RS + i] = 0.0;
+    }
+    for (int i = tid; i < 2 * g.GP; i += NT) sm.gath[i] = 0.0;
     for (int i = tid; i < 4 * Cg * PW; i += NT) sm.pre3[i] = 0.0;   // positions L-1, L-2: no rows beyond L
     for (int i = tid; i < 2 * Cg; i += NT) sm.hbuf[i] = 0;
     if (tid == 0) {
@@ -702,20 +863,40 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         }
     }
-    // One register array holds either the transposed transition weights Er
-    // (transition lanes) or the chain state (owner lanes).
+    // One register array holds the transposed transition weights Er (transition
+    // lanes), the window weights exp(D) of the lane's rows (window lanes, when
+    // they fit) or the chain state (owner lanes).
     // Chain state at the start of step s: V1 = V[s+1], V2 = V[s+2] (reference of
     // s+1) and, prepared from everything but V[s+1]:
     //   pre = V[s+2] W1 + pre3_s, eb = exp(ln2 (rb - kb) - S_s), gg = exp(S_s + ln2 (kb - rb)),
     //   pbe = pre eb, w0e = W0 eb, so bp[s] = V[s+1] w0e + pbe is one FMA after V[s+1];
     //   coef = X[s] (start factor at the reference rb), a2 (transition factor).
-    constexpr int NU = CPL > 14 ? CPL : 14;
+    constexpr int NU = CPL > 16 ? CPL : 16;
+    const int nrw = K > 2 ? (K - 2 + g.LPW - 1) / g.LPW : 0;   // window rows per lane
+    const bool wreg = g.NRB > 0;
     double R[NU];
 #pragma unroll
     for (int m = 0; m < NU; ++m) {
         const int cc = j + m * g.LPL;
-        R[m] = (m < CPL && ro.is_tr && ro.lab_ok && cc < C) ? exp((double)a.A[(size_t)c * C + cc]) : 0.0;
+        double v = 0.0;
+        if (m < CPL && ro.is_tr && ro.lab_ok && cc < C) v = exp((double)a.A[(size_t)c * C + cc]);
+        const int i = 1 + j + m * g.LPW;   // window lanes: row s + i, duration i + 2
+        if (ro.is_win && wreg && ro.lab_ok && m < nrw && i <= K - 2) v = exp((double)a.D[(size_t)(i + 1) * C + c]);
+        R[m] = v;
     }
+    const bool split = CLUSTER && g.NWO == 1 && Cg <= 16 && g.G >= 2;
+    const int slab = split ? (lane & 15) : lc;
+    const bool sends = ro.is_own && slab < cg_own && (split || ro.lab_ok);
+    const int gcnt = split ? g.G / 2 : g.G;
+    // each owner lane's destinations are mapped once into shared memory; a CTA's
+    // shared window maps contiguously, so the mbarrier's mapped address is the
+    // value slot's plus the same offset as locally
+    const uint32_t gloc = smem_addr(&sm.gath[c0l + slab]);
+    uint32_t *rmap = sm.rmap + (size_t)(ro.is_own ? tid : 0) * 16;   // owner threads are 0 .. 32 NWO - 1
+    if (CLUSTER && sends)
+        for (int k = 0; k < gcnt; ++k)
+            rmap[k] = mapa_rank(gloc, (uint32_t)((split && lane >= 16 ? g.G / 2 : 0) + k));
+    const uint32_t bar_off = smem_addr(&sm.full[0]) - gloc;
     double(&Er)[CPL] = *reinterpret_cast<double(*)[CPL]>(&R[0]);
     double &W0 = R[0], &W1 = R[1], &V1 = R[2], &V2 = R[3], &pre = R[4], &gg = R[5], &pbe = R[6], &w0e = R[7],
            &coef = R[8], &a2 = R[9], &mu_acc = R[10], &musum = R[11], &bp = R[12], &start = R[13];
@@ -782,13 +963,21 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
         const int par = u & 1;
         if (ro.is_own) {
             // ------------------------------------------------ owners: chain
-            if (own) {
-                bp = fma(V1, w0e, pbe);
-                if constexpr (CLUSTER) {
-                    for (int g2 = 0; g2 < g.G; ++g2) st_async_f64(&sm.gath[par * C + c], &sm.full[par], g2, bp);
-                } else {
-                    sm.gath[par * C + c] = bp;
+            if (own) bp = fma(V1, w0e, pbe);
+            if constexpr (CLUSTER) {
+                const double sv = split ? __shfl_sync(0xffffffffu, bp, lane & 15) : bp;
+                if (sends) {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        if (k < gcnt) {
+                            const uint32_t ra = rmap[k];
+                            st_async_at(ra + par * g.GP * 8, ra + bar_off + par * 8, sv);
+                        }
                 }
+            } else if (own) {
+                sm.gath[par * g.GP + c] = bp;
+            }
+            if (own) {
                 const double pb = fma(V1, W0, pre);
                 start = coef * pb;   // marginal of a segment of label c starting at s
                 const int ex = exponent_of(pb);
@@ -810,23 +999,6 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
                 cta_arrive(1, NOT);
                 if (g.NWO > 1) cta_barrier(7, 32 * g.NWO);
                 else __syncwarp();
-            }
-            if (warp == 0) {
-                // backward normaliser (the same in every CTA)
-                if (!wait_values<CLUSTER>(sm, par, u, timed_out)) {
-                    timed_out = true;
-                    set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
-                }
-                if constexpr (CLUSTER) cta_arrive(5, NXW);   // bp[s] of every label has arrived
-                const double n = warp_total(sm.gath + par * C, C, lane);
-                if (lane == 0) {
-                    const int kk = sm.kbuf[u & 3];
-                    if (s == 0) {
-                        if (rank == 0) a.logzb[b] = kLn2 * (double)kk + log(n);
-                    } else if (s >= 2) {
-                        sm.kbuf[(u + 2) & 3] = kk + exponent_of(n);
-                    }
-                }
             }
             cta_barrier(4, NOT);
             // ------------------------------------------------ owners: new row
@@ -861,22 +1033,37 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
             }
         } else if (ro.is_tr) {
             // ------------------------------------------- transposed transition
-            if constexpr (CLUSTER) cta_barrier(5, NXW);
-            else cta_barrier(1, NOT);
-            double v[CPL];
-#pragma unroll
-            for (int m = 0; m < CPL; ++m) {
-                const int cc = j + m * g.LPL;
-                v[m] = cc < C ? sm.gath[par * C + cc] : 0.0;
+            if constexpr (CLUSTER) {
+                if (!wait_values<CLUSTER>(sm, par, u, timed_out)) {
+                    timed_out = true;
+                    set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
+                }
+            } else {
+                cta_barrier(1, NOT);
             }
-            const double q = group_sum(tree_dot<CPL>(Er, v), g.LPL);
+            const double *gp = sm.gath + par * g.GP + j;   // zeros past C
+            double vs;
+            const double q = group_sum(chunked_dot<CPL>(gp, g.LPL, Er, &vs), g.LPL);
             if (ro.lab_ok && j == 0) sm.qbuf[lc] = q;
+            // backward normaliser, formed as in the forward (the same in every CTA)
+            const double n = group_sum(vs, g.LPL);
+            if (lc == 0 && j == 0) {
+                const int kk = sm.kbuf[u & 3];
+                if (s == 0) {
+                    if (rank == 0) a.logzb[b] = kLn2 * (double)kk + log(n);
+                } else if (s >= 2) {
+                    sm.kbuf[(u + 2) & 3] = kk + exponent_of(n);
+                }
+            }
             cta_arrive(4, NOT);
         } else if (ro.is_win) {
             // ----------------------- window sums two positions ahead (position s-2)
             if (CLUSTER && tid == W0T) mbar_expect_tx(&sm.full[par], C * 8);
             const int hp = ro.lab_ok ? sm.hbuf[(par ^ 1) * Cg + lc] : 0;   // rebase at s+1
-            const double v = ro.lab_ok ? window_bwd(sm.ring, sm.Wd, K, RS, lc, g.LPW, j, sK, hp) : 0.0;
+            double v = 0.0;
+            if (ro.lab_ok)
+                v = wreg ? window_bwd_nr<NU>(g.NRB, sm.ring, K, RS, lc, g.LPW, j, sK, hp, R)
+                         : window_bwd(sm.ring, sm.Wd, K, RS, lc, g.LPW, j, sK, hp);
             const double sum = group_sum(v, g.LPW < 32 ? g.LPW : 32);
             if (ro.lab_ok && (j & 31) == 0 && s >= 2) sm.pre3[((u + 2) & 3) * Cg * PW + lc * PW + (j >> 5)] = sum;
         }
@@ -1078,11 +1265,13 @@ static bool cl_try(int K, int C, bool bwd, int G, int LPL, int LPW, ClGeom *out,
     if (G > C) return false;
     g.Cg = (C + G - 1) / G;
     if ((G - 1) * g.Cg >= C) return false;   // every CTA owns at least one label
+    if (G > 16) return false;
     g.RS = g.Cg | 1;
     g.LPL = LPL;
     if (LPL < 1 || LPL > 32 || (LPL & (LPL - 1))) return false;
     g.CPL = (C + LPL - 1) / LPL;
     if (g.CPL > 32) return false;
+    g.GP = C > cl_cpl_bucket(g.CPL) * LPL ? C : cl_cpl_bucket(g.CPL) * LPL;
     g.NWO = (g.Cg + 31) / 32;
     g.NWT = (g.Cg * LPL + 31) / 32;
     const int rows = K > 2 ? K - 2 : 1;   // window rows d = 3..K (forward), i = 1..K-2 (backward)
@@ -1091,6 +1280,15 @@ static bool cl_try(int K, int C, bool bwd, int G, int LPL, int LPW, ClGeom *out,
     g.PW = g.LPW > 32 ? g.LPW / 32 : 1;
     g.NWW = (g.Cg * g.LPW + 31) / 32;
     if (g.NWW < 1) g.NWW = 1;
+    // window weights in registers when a lane's rows fit the kernel's register
+    // array (max(CPL bucket, 16) doubles), read in buckets of 8, 16 or 32 rows;
+    // the ring then carries zero rows on both sides for the rows past the window
+    {
+        const int nrw = K > 2 ? (K - 2 + LPW - 1) / LPW : 0;
+        const int nu = cl_cpl_bucket(g.CPL) > 16 ? cl_cpl_bucket(g.CPL) : 16;
+        g.NRB = (nrw > 0 && nrw <= nu) ? (nrw <= 8 ? 8 : nrw <= 16 ? 16 : 32) : 0;
+        g.PAD = g.NRB > 0 && g.NRB * LPW + 2 > K ? g.NRB * LPW + 2 - K : 0;
+    }
     g.NT = 32 * (g.NWO + g.NWT + g.NWW);
     if (g.NT > 1024) return false;
     const int maxt = cl_max_threads(g.NT);
@@ -1117,34 +1315,50 @@ static bool cl_try(int K, int C, bool bwd, int G, int LPL, int LPW, ClGeom *out,
     return true;
 }
 
-// The cheapest geometry by the cost model (ties: the smaller cluster).
+// Every feasible geometry with its cost, cheapest first (ties: the smaller
+// cluster).  Cluster sizes are powers of two; extra = true adds 12 and 14 (the
+// fallbacks when no power of two keeps enough clusters resident at once).
 // SEMICRF_CL_PLAN="G,LPL,LPW" (0 = free choice for that field) restricts the
-// search; the shape is unsupported if nothing fits.
-bool cl_plan(int K, int C, bool bwd, ClGeom *out)
+// search.
+static bool cl_candidates(int K, int C, bool bwd, bool extra, std::vector<std::pair<double, ClGeom>> &out)
 {
     int fG = 0, fL = 0, fW = 0;
     const char *env = getenv("SEMICRF_CL_PLAN");
     if (env && *env && sscanf(env, "%d,%d,%d", &fG, &fL, &fW) < 1) return false;
-    bool found = false;
-    double best = 0.0;
-    for (int G = 1; G <= 16; G *= 2) {
-        if (fG > 0 && G != fG) continue;
+    const int pow2[] = {1, 2, 4, 8, 16}, more[] = {12, 14};
+    const int *Gs = extra ? more : pow2;
+    int nG = extra ? 2 : 5;
+    if (fG > 0) {   // a forced cluster size is taken as given (any of 1..16)
+        if (extra) return true;
+        Gs = &fG;
+        nG = 1;
+    }
+    for (int gi = 0; gi < nG; ++gi) {
+        const int G = Gs[gi];
         for (int LPL = 1; LPL <= 32; LPL *= 2) {
             if (fL > 0 && LPL != fL) continue;
             for (int LPW = 1; LPW <= 256; LPW *= 2) {
                 if (fW > 0 && LPW != fW) continue;
                 ClGeom g;
                 double cost;
-                if (!cl_try(K, C, bwd, G, LPL, LPW, &g, &cost)) continue;
-                if (!found || cost < best) {
-                    best = cost;
-                    *out = g;
-                    found = true;
-                }
+                if (cl_try(K, C, bwd, G, LPL, LPW, &g, &cost)) out.push_back({cost, g});
             }
         }
     }
-    return found;
+    std::stable_sort(out.begin(), out.end(),
+                     [](const std::pair<double, ClGeom> &x, const std::pair<double, ClGeom> &y) {
+                         return x.first < y.first;
+                     });
+    return true;
+}
+
+// The cheapest geometry by the cost model; the shape is unsupported if nothing fits.
+bool cl_plan(int K, int C, bool bwd, ClGeom *out)
+{
+    std::vector<std::pair<double, ClGeom>> c;
+    if (!cl_candidates(K, C, bwd, false, c) || c.empty()) return false;
+    *out = c.front().second;
+    return true;
 }
 
 #define SEMICRF_CL_CASE(CPL, MAXT, CALL) \
@@ -1158,50 +1372,10 @@ bool cl_plan(int K, int C, bool bwd, ClGeom *out)
     SEMICRF_CL_CASE(16, 768, CALL)(__VA_ARGS__); SEMICRF_CL_CASE(32, 256, CALL)(__VA_ARGS__);              \
     SEMICRF_CL_CASE(32, 512, CALL)(__VA_ARGS__);
 
-cudaError_t launch_cl_forward(const FbArgs &a, cudaStream_t st, bool recompute)
+// Clusters of this geometry the current device holds at once (path 0: fused
+// launch, 1: forward, 2: backward), -1 when the query fails.
+static int cl_resident(const ClGeom &g, int K, int C, int path)
 {
-    ClGeom g;
-    if (!cl_plan(a.K, a.C, false, &g)) return cudaErrorInvalidConfiguration;
-    const int cpl = cl_cpl_bucket(g.CPL), maxt = cl_max_threads(g.NT);
-    SEMICRF_CL_TABLE(launch_cl_fwd_tpl, g, a, st, recompute)
-    return cudaErrorInvalidConfiguration;
-}
-
-// One geometry for both chains: the planner's backward plan (its layout is the
-// larger of the two and fits both).
-cudaError_t launch_cl_fused(const FbArgs &a, cudaStream_t st)
-{
-    ClGeom g;
-    if (!cl_plan(a.K, a.C, true, &g)) return cudaErrorInvalidConfiguration;
-    const int cpl = cl_cpl_bucket(g.CPL), maxt = cl_max_threads(g.NT);
-    SEMICRF_CL_TABLE(launch_cl_fused_tpl, g, a, st)
-    return cudaErrorInvalidConfiguration;
-}
-
-cudaError_t launch_cl_backward(const FbArgs &a, cudaStream_t st)
-{
-    ClGeom g;
-    if (!cl_plan(a.K, a.C, true, &g)) return cudaErrorInvalidConfiguration;
-    const int cpl = cl_cpl_bucket(g.CPL), maxt = cl_max_threads(g.NT);
-    SEMICRF_CL_TABLE(launch_cl_bwd_tpl, g, a, st)
-    return cudaErrorInvalidConfiguration;
-}
-#undef SEMICRF_CL_TABLE
-
-// The geometry the planner picks for a path and how many such clusters fit at
-// once: info = {G, NT, Cg, LPL, LPW, shared bytes, resident clusters (-1 when the
-// CUDA query fails, e.g. without a GPU)}.
-bool cl_plan_info(int K, int C, int path, int32_t *info)
-{
-    ClGeom g;
-    if (!cl_plan(K, C, path != 1, &g)) return false;
-    info[0] = g.G;
-    info[1] = g.NT;
-    info[2] = g.Cg;
-    info[3] = g.LPL;
-    info[4] = g.LPW;
-    info[5] = (int32_t)cl_smem_bytes_impl(K, C, g, path != 1);
-    info[6] = -1;
     const int cpl = cl_cpl_bucket(g.CPL), maxt = cl_max_threads(g.NT);
     int n = -1;
     cudaError_t e = cudaErrorInvalidConfiguration;
@@ -1212,11 +1386,112 @@ bool cl_plan_info(int K, int C, int path, int32_t *info)
     SEMICRF_OCC_CASE(16, 256); SEMICRF_OCC_CASE(16, 512); SEMICRF_OCC_CASE(16, 768);
     SEMICRF_OCC_CASE(32, 256); SEMICRF_OCC_CASE(32, 512);
 #undef SEMICRF_OCC_CASE
-    if (e == cudaSuccess) info[6] = n;
-    else cudaGetLastError();   // clear a failed query
+    if (e != cudaSuccess) {
+        cudaGetLastError();   // clear a failed query
+        return -1;
+    }
+    return n;
+}
+
+// The geometry a launch of `need` concurrent clusters uses: the cheapest one of
+// which the device holds `need` clusters at once (all chains of the launch then
+// run side by side), trying the power-of-two cluster sizes first and 12 and 14
+// after; if none does, the cheapest.  Cached per device and shape.
+static bool cl_plan_resident(int K, int C, int path, int need, ClGeom *out)
+{
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int, int, int>, ClGeom> cache;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        dev = -1;
+    }
+    const char *env = getenv("SEMICRF_CL_PLAN");
+    const bool forced = env && *env;
+    const auto key = std::make_tuple(K, C, path, need, dev);
+    if (!forced) {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find(key);
+        if (it != cache.end()) {
+            *out = it->second;
+            return true;
+        }
+    }
+    const bool bwd = path != 1;
+    std::vector<std::pair<double, ClGeom>> c;
+    if (!cl_candidates(K, C, bwd, false, c) || c.empty()) return false;
+    ClGeom pick = c.front().second;
+    bool ok = forced || dev < 0 || need <= 1 || cl_resident(pick, K, C, path) >= need;
+    for (size_t i = 1; !ok && i < c.size(); ++i)
+        if (cl_resident(c[i].second, K, C, path) >= need) {
+            pick = c[i].second;
+            ok = true;
+        }
+    if (!ok) {
+        std::vector<std::pair<double, ClGeom>> x;
+        cl_candidates(K, C, bwd, true, x);
+        for (size_t i = 0; !ok && i < x.size(); ++i)
+            if (cl_resident(x[i].second, K, C, path) >= need) {
+                pick = x[i].second;
+                ok = true;
+            }
+    }
+    *out = pick;
+    if (!forced) {
+        std::lock_guard<std::mutex> lock(mu);
+        cache[key] = pick;
+    }
     return true;
 }
 
+cudaError_t launch_cl_forward(const FbArgs &a, cudaStream_t st, bool recompute)
+{
+    ClGeom g;
+    // the checkpoint recompute launches B*J clusters that queue by design
+    if (!(recompute ? cl_plan(a.K, a.C, false, &g) : cl_plan_resident(a.K, a.C, 1, a.B, &g)))
+        return cudaErrorInvalidConfiguration;
+    const int cpl = cl_cpl_bucket(g.CPL), maxt = cl_max_threads(g.NT);
+    SEMICRF_CL_TABLE(launch_cl_fwd_tpl, g, a, st, recompute)
+    return cudaErrorInvalidConfiguration;
+}
+
+// One geometry for both chains (the backward layout is the larger of the two and
+// fits both), chosen so that all 2B chains are resident at once when possible.
+cudaError_t launch_cl_fused(const FbArgs &a, cudaStream_t st)
+{
+    ClGeom g;
+    if (!cl_plan_resident(a.K, a.C, 0, 2 * a.B, &g)) return cudaErrorInvalidConfiguration;
+    const int cpl = cl_cpl_bucket(g.CPL), maxt = cl_max_threads(g.NT);
+    SEMICRF_CL_TABLE(launch_cl_fused_tpl, g, a, st)
+    return cudaErrorInvalidConfiguration;
+}
+
+cudaError_t launch_cl_backward(const FbArgs &a, cudaStream_t st)
+{
+    ClGeom g;
+    if (!cl_plan_resident(a.K, a.C, 2, a.B, &g)) return cudaErrorInvalidConfiguration;
+    const int cpl = cl_cpl_bucket(g.CPL), maxt = cl_max_threads(g.NT);
+    SEMICRF_CL_TABLE(launch_cl_bwd_tpl, g, a, st)
+    return cudaErrorInvalidConfiguration;
+}
+#undef SEMICRF_CL_TABLE
+
+// The geometry a launch of B sequences uses for a path and how many such
+// clusters fit at once: info = {G, NT, Cg, LPL, LPW, shared bytes, resident
+// clusters (-1 when the CUDA query fails, e.g. without a GPU)}.
+bool cl_plan_info(int K, int C, int B, int path, int32_t *info)
+{
+    ClGeom g;
+    if (!cl_plan_resident(K, C, path, path == 0 ? 2 * B : B, &g)) return false;
+    info[0] = g.G;
+    info[1] = g.NT;
+    info[2] = g.Cg;
+    info[3] = g.LPL;
+    info[4] = g.LPW;
+    info[5] = (int32_t)cl_smem_bytes_impl(K, C, g, path != 1);
+    info[6] = cl_resident(g, K, C, path);
+    return true;
+}
 
 #undef SEMICRF_CL_CASE
 

@@ -175,13 +175,16 @@ using namespace semicrf;
 
 namespace {
 
-semicrf_status check_dims_impl(const semicrf_dims *d)
+// chains = false: the prefix scan alone, which runs no chain kernel (its dims
+// carry K = 1), so no chain geometry is required.
+semicrf_status check_dims_impl(const semicrf_dims *d, bool chains = true)
 {
     if (!d) return SEMICRF_ERR_INVALID_ARG;
     if (d->B < 1 || d->T < 1 || d->K < 1 || d->C < 1 || d->ckpt_interval < 0)
         return SEMICRF_ERR_INVALID_ARG;
     if (d->C > SEMICRF_MAX_C || d->K > SEMICRF_MAX_K) return SEMICRF_ERR_UNSUPPORTED_SHAPE;
     if ((long long)d->B * (d->T + 1) * d->C > (1LL << 40)) return SEMICRF_ERR_UNSUPPORTED_SHAPE;
+    if (!chains) return SEMICRF_OK;
     if (!make_plan(d->K, d->C).ok()) return SEMICRF_ERR_UNSUPPORTED_SHAPE;   // Viterbi layout
     if (!small_path_ok(d->K, d->C)) {
         ClGeom g;
@@ -195,7 +198,7 @@ semicrf_status prepare(const semicrf_dims *d, int what, void *ws, size_t ws_byte
                        Layout *lay)
 {
     prof_reset();
-    semicrf_status s = check_dims_impl(d);
+    semicrf_status s = check_dims_impl(d, what != SEMICRF_WS_SCAN);
     if (s != SEMICRF_OK) return s;
     if (!ws) return SEMICRF_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return SEMICRF_ERR_INVALID_ARG;
@@ -267,7 +270,7 @@ semicrf_status semicrf_check_dims(const semicrf_dims *dims) { return check_dims_
 
 size_t semicrf_workspace_bytes(const semicrf_dims *dims, int32_t what)
 {
-    if (check_dims_impl(dims) != SEMICRF_OK) return 0;
+    if (check_dims_impl(dims, what != SEMICRF_WS_SCAN) != SEMICRF_OK) return 0;
     Plan p = make_plan(dims->K, dims->C);
     Layout lay;
     if (!make_layout(*dims, what, p, &lay)) return 0;
@@ -661,7 +664,7 @@ semicrf_status semicrf_chain_plan(const semicrf_dims *dims, int32_t path, int32_
         return SEMICRF_OK;
     }
     info[0] = 1;
-    if (!cl_plan_info(dims->K, dims->C, path, info + 1)) return SEMICRF_ERR_UNSUPPORTED_SHAPE;
+    if (!cl_plan_info(dims->K, dims->C, dims->B, path, info + 1)) return SEMICRF_ERR_UNSUPPORTED_SHAPE;
     info[8] = path == 0 ? 2 * dims->B : dims->B;
     return SEMICRF_OK;
 }

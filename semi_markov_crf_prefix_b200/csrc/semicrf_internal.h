@@ -142,9 +142,14 @@ struct FbArgs {
 // when LPW > 32).
 // RS is the shared-memory row stride (doubles) of the ring, duration-weight and
 // duration-accumulator arrays: odd, so that the lanes of one label, which read
-// consecutive rows, fall in different banks.
+// consecutive rows, fall in different banks.  GP is the pitch of the exchanged
+// values (>= C, zeros past C, so the transition lanes read without bounds).
+// NRB: rows per window lane read with the weights in registers (8, 16 or 32;
+// 0: the weights stay in shared memory); PAD: zero ring rows before and after
+// the ring for the rows a window lane reads past the window.
 struct ClGeom {
-    int G = 0, Cg = 0, LPL = 0, CPL = 0, LPW = 0, PW = 0, NWO = 0, NWT = 0, NWW = 0, NT = 0, RS = 0;
+    int G = 0, Cg = 0, LPL = 0, CPL = 0, LPW = 0, PW = 0, NWO = 0, NWT = 0, NWW = 0, NT = 0, RS = 0, GP = 0;
+    int NRB = 0, PAD = 0;
 };
 bool cl_plan(int K, int C, bool bwd, ClGeom *out);
 cudaError_t launch_cl_forward(const FbArgs &a, cudaStream_t st, bool recompute);
@@ -153,7 +158,7 @@ cudaError_t launch_cl_backward(const FbArgs &a, cudaStream_t st);
 cudaError_t launch_cl_fused(const FbArgs &a, cudaStream_t st);
 // Planner's choice for path 0 (fused), 1 (forward) or 2 (backward) and how many
 // such clusters the GPU holds at once (see semicrf_chain_plan).
-bool cl_plan_info(int K, int C, int path, int32_t *info);
+bool cl_plan_info(int K, int C, int B, int path, int32_t *info);
 // dD and dA from the cluster backward's stored rows (cl_grads.cu): two contraction
 // kernels writing split partial sums, one kernel reducing them (3 launches).
 constexpr int kGradChunk = 64;   // start positions per staged chunk
