@@ -178,6 +178,7 @@ def test_nll_entry_points():
     dX, dA, dD = sc.nll_backward(S, A, D, lens, lb, sg, ws, grad_nll=g)
     assert sc.device_status(ws) == 0
     ws2 = sc.new_workspace(w.B, w.T, w.K, w.C, sc.WS_TRAIN, device=dev)
+    sc.clear_device_status(ws2)
     logZ2, _ = sc.forward(S, A, D, lens, ws=ws2)
     score2 = sc.gold_score(S, A, D, lens, lb, sg, ws2)
     rX, rA, rD = sc.backward(S, A, D, lens, ws2, grad_logZ=g)
