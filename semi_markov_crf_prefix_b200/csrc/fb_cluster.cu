@@ -7,18 +7,22 @@
 // summary 2.A-2.C).  A CTA has three kinds of warps.  Owner warps run the chain
 // of one label per lane; transition warps form the C x C product; window warps
 // form the duration sums.  The sequential chain of one position is
-//   owners:      p = U[t-1] W0 + pre_t ;  a'[t,c] = p e ; st.async of a'[t,c]
-//                into every CTA of the cluster, completing bytes on that CTA's
-//                mbarrier for the position (G = 1: a plain store + bar.arrive)
-//   transition:  wait for the C values, q[c] = sum_c' a'[t,c'] exp(A[c',c])
-//                (LPL lanes per label, CPL terms each, shuffle reduction; the
-//                same pass sums n_t = sum_c' a'[t,c'] for the normaliser);
-//                bar.arrive to the owners
+//   owners:      p = U[t-1] W0 + pre_t ;  a'[t,c] = p e into a stage buffer;
+//                one bulk copy of the CTA's block of values (cp.async.bulk,
+//                shared::cta to shared::cluster, no multicast) to every CTA of
+//                the cluster, completing its bytes on that CTA's mbarrier for
+//                the position (G = 1: a plain store + bar.arrive)
+//   transition:  wait on the mbarrier, q[c] = sum_c' a'[t,c'] exp(A[c',c])
+//                (LPL lanes per label, CPL terms each, shuffle reduction);
+//                bar.arrive to the owners; the lanes of the first label then
+//                sum n_t = sum_c' a'[t,c'] for the normaliser
 //   owners:      bar.sync, U[t,c] = q f, the new ring row
 //   all:         one bar.sync (with an OR of the timeout flags) per position
 // Work off the chain:
 //  * window warps form the duration sum over d >= 3 two positions ahead,
 //      pre3_{t+2} = sum_{d=3..K} U[t+2-d] exp(D[d-1]),
+//    with their weights exp(D) in registers when their rows fit (8, 16 or 32
+//    per lane; zero rows around the ring stand in for the rows past the window),
 //    starting right after the previous position's barrier, in parallel with
 //    the owners and the exchange.  They read the rows at the reference of
 //    position t-1 and bring them there themselves (a rebase of a column at t-1
@@ -44,6 +48,7 @@
 #include <stdint.h>
 #include <stdio.h>
 #include <stdlib.h>
+#include <string.h>
 
 #include <algorithm>
 #include <map>
@@ -131,12 +136,36 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
     }
 }
 
-// st.async of v to the shared::cluster address ra, completing 8 bytes on the
-// mbarrier at the shared::cluster address rb (both from mapa, done once).
-__device__ __forceinline__ void st_async_at(uint32_t ra, uint32_t rb, double v)
+// group_sum of two values at once (the same order for each as group_sum)
+__device__ __forceinline__ void group_sum2(double &v, double &w, int width)
 {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];" ::"r"(ra),
-                 "l"(__double_as_longlong(v)), "r"(rb)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        if (off < width) {
+            v += __shfl_xor_sync(0xffffffffu, v, off);
+            w += __shfl_xor_sync(0xffffffffu, w, off);
+        }
+}
+
+// The label whose value sits at position i of the exchange buffer (CTA r's Cg
+// labels at r*CgE ..., CgE = Cg rounded up to even; with one CTA the labels in
+// order), or -1 for a padding position.
+__host__ __device__ __forceinline__ int exch_label(int i, int C, int Cg, int G)
+{
+    if (G <= 1) return i < C ? i : -1;
+    const int CgE = (Cg + 1) & ~1;
+    const int r = i / CgE, o = i - r * CgE;
+    const int lab = r * Cg + o;
+    return (o < Cg && r < G && lab < C) ? lab : -1;
+}
+
+// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory at src to
+// the shared::cluster address dst, completing the bytes on the mbarrier at the
+// shared::cluster address bar (both 16-byte aligned; no multicast).
+__device__ __forceinline__ void bulk_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "r"(src), "r"(bytes), "r"(bar)
                  : "memory");
 }
 
@@ -164,7 +193,9 @@ __device__ __forceinline__ double rescale(double x, int h) { return h == 0 ? x :
 struct ClSmem {
     double *ring;    // [2K][RS] every row twice, with LPW zero rows before and after
     double *Wd;      // [K][RS]  exp(D), when the window lanes do not hold it in registers
-    double *gath;    // [2][GP]  a' (forward) or bp (backward) of the position, all labels (zeros past C)
+    double *gath;    // [2][GP]  a' (forward) or bp (backward) of the position: CTA r's labels at
+                     //          positions r*CgE .. r*CgE + Cg - 1 (CgE = Cg rounded up to even), zeros elsewhere
+    double *stage;   // [2][CgE] this CTA's values of the position, the source of the bulk copies
     double *qbuf;    // [Cg]     transition result of each label, for its owner
     double *pre3;    // [4][Cg][PW] window sums two positions ahead
     double *pf_es, *pf_ies, *pf_cu, *pf_ca;   // [kPF][Cg] prefetch rings
@@ -172,15 +203,23 @@ struct ClSmem {
     int *pf_m, *pf_eu, *pf_ea;                // [kPF][Cg] each
     int *hbuf;       // [2][Cg] rebase exponent of each label at the last two positions
     int *kbuf;       // [4]     normaliser exponents
-    uint32_t *rmap;  // [32*NWO][16] mapped destination of each owner lane's value, per CTA of the cluster
 };
+
+__host__ __device__ __forceinline__ size_t even_up(size_t n) { return (n + 1) & ~(size_t)1; }
+
+// Doubles before the exchange buffers (rounded up to an even count, so that the
+// exchange buffers start on a 16-byte boundary, as bulk copies require).
+__host__ __device__ __forceinline__ size_t cl_head_doubles(int K, const ClGeom &g)
+{
+    return even_up(((g.NRB > 0 ? 2 : 3) * (size_t)K + 2 * (size_t)g.PAD) * g.RS);
+}
 
 __host__ __device__ __forceinline__ size_t cl_smem_bytes_impl(int K, int C, const ClGeom &g, bool bwd)
 {
     const size_t npf = bwd ? 4 : 2;
-    const size_t nd = ((g.NRB > 0 ? 2 : 3) * (size_t)K + 2 * (size_t)g.PAD) * g.RS + 2 * (size_t)g.GP + g.Cg +
+    const size_t nd = cl_head_doubles(K, g) + 2 * (size_t)g.GP + 2 * even_up(g.Cg) + even_up(g.Cg) +
                       4 * (size_t)g.Cg * g.PW + npf * kPF * g.Cg;
-    const size_t ni = (bwd ? 3 : 1) * (size_t)kPF * g.Cg + 2 * (size_t)g.Cg + 4 + 32 * 16 * (size_t)g.NWO;
+    const size_t ni = (bwd ? 3 : 1) * (size_t)kPF * g.Cg + 2 * (size_t)g.Cg + 4;
     return nd * sizeof(double) + 2 * sizeof(uint64_t) + ni * sizeof(int);
 }
 
@@ -189,9 +228,10 @@ __device__ __forceinline__ ClSmem cl_smem(double *base, int K, int C, const ClGe
     ClSmem s;
     s.ring = base + (size_t)g.PAD * g.RS;
     s.Wd = s.ring + (2 * (size_t)K + g.PAD) * g.RS;
-    s.gath = s.Wd + (g.NRB > 0 ? 0 : (size_t)K * g.RS);
-    s.qbuf = s.gath + 2 * (size_t)g.GP;
-    s.pre3 = s.qbuf + g.Cg;
+    s.gath = base + cl_head_doubles(K, g);
+    s.stage = s.gath + 2 * (size_t)g.GP;
+    s.qbuf = s.stage + 2 * even_up(g.Cg);
+    s.pre3 = s.qbuf + even_up(g.Cg);
     s.pf_es = s.pre3 + 4 * g.Cg * g.PW;
     s.pf_ies = s.pf_es + kPF * g.Cg;
     s.pf_cu = s.pf_ies + kPF * g.Cg;
@@ -203,7 +243,6 @@ __device__ __forceinline__ ClSmem cl_smem(double *base, int K, int C, const ClGe
     s.pf_ea = bwd ? s.pf_eu + kPF * g.Cg : s.pf_eu;
     s.hbuf = bwd ? s.pf_ea + kPF * g.Cg : s.pf_eu;
     s.kbuf = s.hbuf + 2 * g.Cg;
-    s.rmap = reinterpret_cast<uint32_t *>(s.kbuf + 4);
     return s;
 }
 
@@ -305,16 +344,22 @@ __device__ __forceinline__ double window_fwd_reg(double *ring, int K, int RS, in
 {
     static_assert(NR <= NU, "window rows exceed the register array");
     const int d0 = 3 + j;
-    if (hp != 0 && d0 <= K) {
-        const int n = (K - d0) / LPW + 1;
-        for (int m = 0; m < n; ++m) {
+    if (hp != 0) {
+        // a rebase at tau - 3 (every label rebases about every 500 bits of growth of
+        // its column, and the labels of a chain within a few positions of each
+        // other): the lane's rows d >= 4 of the window, both copies, times the
+        // exact power of two
+        const double s2a = pow2c(hp / 2), s2b = pow2c(hp - hp / 2);   // as scale2c
+#pragma unroll 4
+        for (int m = 0; m < NR; ++m) {
             const int d = d0 + m * LPW;
-            if (d < 4) continue;
-            const int sl = tauK + K - d;
-            const int other = sl >= K ? sl - K : sl + K;
-            const double v = rescale(ring[sl * RS + lc], hp);
-            ring[sl * RS + lc] = v;
-            ring[other * RS + lc] = v;
+            if (d >= 4 && d <= K) {
+                const int sl = tauK + K - d;
+                const int other = sl >= K ? sl - K : sl + K;
+                const double v = (ring[sl * RS + lc] * s2a) * s2b;
+                ring[sl * RS + lc] = v;
+                ring[other * RS + lc] = v;
+            }
         }
     }
     const double *p = ring + (tauK + K - d0) * RS + lc;
@@ -331,16 +376,18 @@ __device__ __forceinline__ double window_bwd_reg(double *ring, int K, int RS, in
 {
     static_assert(NR <= NU, "window rows exceed the register array");
     const int i0 = 1 + j;
-    if (hp != 0 && i0 <= K - 2) {
-        const int n = (K - 2 - i0) / LPW + 1;
-        for (int m = 0; m < n; ++m) {
+    if (hp != 0) {
+        const double s2a = pow2c(hp / 2), s2b = pow2c(hp - hp / 2);   // as in the forward: rows i >= 2
+#pragma unroll 4
+        for (int m = 0; m < NR; ++m) {
             const int i = i0 + m * LPW;
-            if (i < 2) continue;
-            const int sl = sK + i;
-            const int other = sl >= K ? sl - K : sl + K;
-            const double v = rescale(ring[sl * RS + lc], hp);
-            ring[sl * RS + lc] = v;
-            ring[other * RS + lc] = v;
+            if (i >= 2 && i <= K - 2) {
+                const int sl = sK + i;
+                const int other = sl >= K ? sl - K : sl + K;
+                const double v = (ring[sl * RS + lc] * s2a) * s2b;
+                ring[sl * RS + lc] = v;
+                ring[other * RS + lc] = v;
+            }
         }
     }
     const double *p = ring + (sK + i0) * RS + lc;
@@ -531,6 +578,7 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
             sm.ring[2 * K * RS + i] = 0.0;
         }
         for (int i = tid; i < 2 * g.GP; i += NT) sm.gath[i] = 0.0;
+        for (int i = tid; i < 2 * (int)even_up(Cg); i += NT) sm.stage[i] = 0.0;
         for (int i = tid; i < 4 * Cg * PW; i += NT) sm.pre3[i] = 0.0;
         for (int i = tid; i < 2 * Cg; i += NT) sm.hbuf[i] = 0;
         if (tid == 0) {
@@ -575,7 +623,8 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
     for (int m = 0; m < NU; ++m) {
         const int cp = j + m * g.LPL;
         double v = 0.0;
-        if (m < CPL && ro.is_tr && ro.lab_ok && cp < C) v = exp((double)a.A[(size_t)cp * C + c]);
+        const int lp = exch_label(cp, C, Cg, g.G);   // the label at exchange position cp, or -1
+        if (m < CPL && ro.is_tr && ro.lab_ok && lp >= 0) v = exp((double)a.A[(size_t)lp * C + c]);
         const int d = 3 + j + m * g.LPW;   // window lanes: duration of row m
         if (ro.is_win && wreg && ro.lab_ok && m < nrw && d <= K) v = exp((double)a.D[(size_t)(d - 1) * C + c]);
         R[m] = v;
@@ -592,23 +641,14 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
             if (ro.lab_ok && (j & 31) == 0) sm.pre3[(q - 1) * Cg * PW + lc * PW + (j >> 5)] = s;
         }
     }
-    // The exchange: each owner label's value goes to every CTA of the cluster.
-    // With one owner warp and at most 16 labels per CTA the warp's upper half
-    // sends the upper half of the ranks (the value shuffled from the lower half).
-    // Destination addresses are mapped once.
-    const bool split = CLUSTER && g.NWO == 1 && Cg <= 16 && g.G >= 2;
-    const int slab = split ? (lane & 15) : lc;
-    const bool sends = ro.is_own && slab < cg_own && (split || ro.lab_ok);
-    const int gcnt = split ? g.G / 2 : g.G;
-    // each owner lane's destinations are mapped once into shared memory; a CTA's
-    // shared window maps contiguously, so the mbarrier's mapped address is the
-    // value slot's plus the same offset as locally
-    const uint32_t gloc = smem_addr(&sm.gath[c0l + slab]);
-    uint32_t *rmap = sm.rmap + (size_t)(ro.is_own ? tid : 0) * 16;   // owner threads are 0 .. 32 NWO - 1
-    if (CLUSTER && sends)
-        for (int k = 0; k < gcnt; ++k)
-            rmap[k] = mapa_rank(gloc, (uint32_t)((split && lane >= 16 ? g.G / 2 : 0) + k));
-    const uint32_t bar_off = smem_addr(&sm.full[0]) - gloc;
+    // The exchange: each CTA's block of values (its labels, padded with zeros to an
+    // even count CgE, so 16-byte units) goes to every CTA of the cluster by one bulk
+    // copy per destination, issued by lane k of warp 0 for CTA k, into position
+    // rank*CgE of the destination's exchange buffer, completing on its mbarrier.
+    const int CgE = (int)even_up(Cg);
+    const bool issuer = CLUSTER && warp == 0 && lane < g.G;
+    const uint32_t bdst = issuer ? mapa_rank(smem_addr(&sm.gath[rank * CgE]), (uint32_t)lane) : 0u;
+    const uint32_t bbar = issuer ? mapa_rank(smem_addr(&sm.full[0]), (uint32_t)lane) : 0u;
     double(&E)[CPL] = *reinterpret_cast<double(*)[CPL]>(&R[0]);
     double &W0 = R[0], &W1 = R[1], &U1 = R[2], &U2 = R[3], &pre = R[4], &f = R[5], &pe = R[6], &w0e = R[7],
            &ap = R[8];
@@ -669,15 +709,15 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
             // ------------------------------------------------ owners: chain
             if (own) ap = fma(U1, w0e, pe);
             if constexpr (CLUSTER) {
-                const double sv = split ? __shfl_sync(0xffffffffu, ap, lane & 15) : ap;
-                if (sends) {
-#pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        if (k < gcnt) {
-                            const uint32_t ra = rmap[k];
-                            st_async_at(ra + par * g.GP * 8, ra + bar_off + par * 8, sv);
-                        }
-                }
+                // the owners' values into the stage, visible to the copy engine, then one
+                // bulk copy per destination CTA
+                if (own) sm.stage[par * CgE + lc] = ap;
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                if (g.NWO > 1) cta_barrier(7, 32 * g.NWO);
+                else __syncwarp();
+                if (issuer)
+                    bulk_to_peer(bdst + par * g.GP * 8, smem_addr(sm.stage + par * CgE), (uint32_t)(CgE * 8),
+                                 bbar + par * 8);
             } else if (own) {
                 sm.gath[par * g.GP + c] = ap;
             }
@@ -738,12 +778,14 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
                 cta_barrier(1, NOT);
             }
             const double *gp = sm.gath + par * g.GP + j;   // zeros past C
-            double vs;
-            const double q = group_sum(chunked_dot<CPL>(gp, g.LPL, E, &vs), g.LPL);
+            // q, and the normaliser n_t = sum_c a'[t,c] from the values the lanes loaded
+            // (the same order in every CTA); n is needed two positions later, so it is
+            // stored after the arrival that releases the owners
+            double n;
+            double q = chunked_dot<CPL>(gp, g.LPL, E, &n);
+            group_sum2(q, n, g.LPL);
             if (ro.lab_ok && j == 0) sm.qbuf[lc] = q;
-            // normaliser n_t = sum_c a'[t,c]: the lanes of the first label sum the values
-            // they loaded, in the same order in every CTA
-            const double n = group_sum(vs, g.LPL);
+            cta_arrive(4, NOT);
             if (lc == 0 && j == 0) {
                 const int kk = sm.kbuf[u & 3];
                 if (t == L) {
@@ -758,10 +800,9 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
                     sm.kbuf[(u + 2) & 3] = kk + exponent_of(n);
                 }
             }
-            cta_arrive(4, NOT);
         } else if (ro.is_win) {
             // ------------------------------------- window sums two positions ahead
-            if (CLUSTER && tid == W0T) mbar_expect_tx(&sm.full[par], C * 8);
+            if (CLUSTER && tid == W0T) mbar_expect_tx(&sm.full[par], g.G * (int)even_up(Cg) * 8);
             const int hp = ro.lab_ok ? sm.hbuf[(par ^ 1) * Cg + lc] : 0;   // rebase at t-1
             const int tau2K = tK + 2 >= K ? tK + 2 - K : tK + 2;   // K >= 3 whenever a row is read
             double v = 0.0;
@@ -852,6 +893,7 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
         sm.ring[2 * K * RS + i] = 0.0;
     }
     for (int i = tid; i < 2 * g.GP; i += NT) sm.gath[i] = 0.0;
+    for (int i = tid; i < 2 * (int)even_up(Cg); i += NT) sm.stage[i] = 0.0;
     for (int i = tid; i < 4 * Cg * PW; i += NT) sm.pre3[i] = 0.0;   // positions L-1, L-2: no rows beyond L
     for (int i = tid; i < 2 * Cg; i += NT) sm.hbuf[i] = 0;
     if (tid == 0) {
@@ -879,24 +921,20 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
     for (int m = 0; m < NU; ++m) {
         const int cc = j + m * g.LPL;
         double v = 0.0;
-        if (m < CPL && ro.is_tr && ro.lab_ok && cc < C) v = exp((double)a.A[(size_t)c * C + cc]);
+        const int lp = exch_label(cc, C, Cg, g.G);
+        if (m < CPL && ro.is_tr && ro.lab_ok && lp >= 0) v = exp((double)a.A[(size_t)c * C + lp]);
         const int i = 1 + j + m * g.LPW;   // window lanes: row s + i, duration i + 2
         if (ro.is_win && wreg && ro.lab_ok && m < nrw && i <= K - 2) v = exp((double)a.D[(size_t)(i + 1) * C + c]);
         R[m] = v;
     }
-    const bool split = CLUSTER && g.NWO == 1 && Cg <= 16 && g.G >= 2;
-    const int slab = split ? (lane & 15) : lc;
-    const bool sends = ro.is_own && slab < cg_own && (split || ro.lab_ok);
-    const int gcnt = split ? g.G / 2 : g.G;
-    // each owner lane's destinations are mapped once into shared memory; a CTA's
-    // shared window maps contiguously, so the mbarrier's mapped address is the
-    // value slot's plus the same offset as locally
-    const uint32_t gloc = smem_addr(&sm.gath[c0l + slab]);
-    uint32_t *rmap = sm.rmap + (size_t)(ro.is_own ? tid : 0) * 16;   // owner threads are 0 .. 32 NWO - 1
-    if (CLUSTER && sends)
-        for (int k = 0; k < gcnt; ++k)
-            rmap[k] = mapa_rank(gloc, (uint32_t)((split && lane >= 16 ? g.G / 2 : 0) + k));
-    const uint32_t bar_off = smem_addr(&sm.full[0]) - gloc;
+    // The exchange: each CTA's block of values (its labels, padded with zeros to an
+    // even count CgE, so 16-byte units) goes to every CTA of the cluster by one bulk
+    // copy per destination, issued by lane k of warp 0 for CTA k, into position
+    // rank*CgE of the destination's exchange buffer, completing on its mbarrier.
+    const int CgE = (int)even_up(Cg);
+    const bool issuer = CLUSTER && warp == 0 && lane < g.G;
+    const uint32_t bdst = issuer ? mapa_rank(smem_addr(&sm.gath[rank * CgE]), (uint32_t)lane) : 0u;
+    const uint32_t bbar = issuer ? mapa_rank(smem_addr(&sm.full[0]), (uint32_t)lane) : 0u;
     double(&Er)[CPL] = *reinterpret_cast<double(*)[CPL]>(&R[0]);
     double &W0 = R[0], &W1 = R[1], &V1 = R[2], &V2 = R[3], &pre = R[4], &gg = R[5], &pbe = R[6], &w0e = R[7],
            &coef = R[8], &a2 = R[9], &mu_acc = R[10], &musum = R[11], &bp = R[12], &start = R[13];
@@ -965,15 +1003,13 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
             // ------------------------------------------------ owners: chain
             if (own) bp = fma(V1, w0e, pbe);
             if constexpr (CLUSTER) {
-                const double sv = split ? __shfl_sync(0xffffffffu, bp, lane & 15) : bp;
-                if (sends) {
-#pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        if (k < gcnt) {
-                            const uint32_t ra = rmap[k];
-                            st_async_at(ra + par * g.GP * 8, ra + bar_off + par * 8, sv);
-                        }
-                }
+                if (own) sm.stage[par * CgE + lc] = bp;   // as in the forward
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                if (g.NWO > 1) cta_barrier(7, 32 * g.NWO);
+                else __syncwarp();
+                if (issuer)
+                    bulk_to_peer(bdst + par * g.GP * 8, smem_addr(sm.stage + par * CgE), (uint32_t)(CgE * 8),
+                                 bbar + par * 8);
             } else if (own) {
                 sm.gath[par * g.GP + c] = bp;
             }
@@ -1042,11 +1078,12 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
                 cta_barrier(1, NOT);
             }
             const double *gp = sm.gath + par * g.GP + j;   // zeros past C
-            double vs;
-            const double q = group_sum(chunked_dot<CPL>(gp, g.LPL, Er, &vs), g.LPL);
+            // q and the backward normaliser, formed as in the forward
+            double n;
+            double q = chunked_dot<CPL>(gp, g.LPL, Er, &n);
+            group_sum2(q, n, g.LPL);
             if (ro.lab_ok && j == 0) sm.qbuf[lc] = q;
-            // backward normaliser, formed as in the forward (the same in every CTA)
-            const double n = group_sum(vs, g.LPL);
+            cta_arrive(4, NOT);
             if (lc == 0 && j == 0) {
                 const int kk = sm.kbuf[u & 3];
                 if (s == 0) {
@@ -1055,10 +1092,9 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
                     sm.kbuf[(u + 2) & 3] = kk + exponent_of(n);
                 }
             }
-            cta_arrive(4, NOT);
         } else if (ro.is_win) {
             // ----------------------- window sums two positions ahead (position s-2)
-            if (CLUSTER && tid == W0T) mbar_expect_tx(&sm.full[par], C * 8);
+            if (CLUSTER && tid == W0T) mbar_expect_tx(&sm.full[par], g.G * (int)even_up(Cg) * 8);
             const int hp = ro.lab_ok ? sm.hbuf[(par ^ 1) * Cg + lc] : 0;   // rebase at s+1
             double v = 0.0;
             if (ro.lab_ok)
@@ -1269,9 +1305,11 @@ static bool cl_try(int K, int C, bool bwd, int G, int LPL, int LPW, ClGeom *out,
     g.RS = g.Cg | 1;
     g.LPL = LPL;
     if (LPL < 1 || LPL > 32 || (LPL & (LPL - 1))) return false;
-    g.CPL = (C + LPL - 1) / LPL;
+    const int npos = G > 1 ? G * (int)even_up(g.Cg) : C;   // exchange positions (labels plus padding)
+    g.CPL = (npos + LPL - 1) / LPL;
     if (g.CPL > 32) return false;
-    g.GP = C > cl_cpl_bucket(g.CPL) * LPL ? C : cl_cpl_bucket(g.CPL) * LPL;
+    g.GP = (int)even_up((size_t)(npos > cl_cpl_bucket(g.CPL) * LPL ? npos : cl_cpl_bucket(g.CPL) * LPL));
+
     g.NWO = (g.Cg + 31) / 32;
     g.NWT = (g.Cg * LPL + 31) / 32;
     const int rows = K > 2 ? K - 2 : 1;   // window rows d = 3..K (forward), i = 1..K-2 (backward)

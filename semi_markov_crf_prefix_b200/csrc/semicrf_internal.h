@@ -143,7 +143,9 @@ struct FbArgs {
 // RS is the shared-memory row stride (doubles) of the ring, duration-weight and
 // duration-accumulator arrays: odd, so that the lanes of one label, which read
 // consecutive rows, fall in different banks.  GP is the pitch of the exchanged
-// values (>= C, zeros past C, so the transition lanes read without bounds).
+// values: G blocks of Cg labels each padded to an even count (16-byte units for
+// the bulk copies), zeros in the padding and past the last block, at least the
+// positions the transition lanes read, so they read without bounds tests.
 // NRB: rows per window lane read with the weights in registers (8, 16 or 32;
 // 0: the weights stay in shared memory); PAD: zero ring rows before and after
 // the ring for the rows a window lane reads past the window.

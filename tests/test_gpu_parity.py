@@ -177,22 +177,24 @@ def test_cluster_geometries(plan, monkeypatch):
         check_against_oracle(w, run_gpu(w))
 
 
-@pytest.mark.parametrize("plan", ["12,0,0", "14,0,0", "14,8,16", "16,8,16"])
+@pytest.mark.parametrize("plan", ["12,0,0", "14,0,0", "16,8,16"])
 def test_cluster_sizes_beyond_powers_of_two(plan, monkeypatch):
-    # clusters of 12 and 14 CTAs (the planner's fallback when 16-CTA clusters
-    # cannot all be resident) on a small random problem, and 14 and 16 at the
-    # large-label workload's K and C on a short sequence (12 does not fit it)
+    # clusters of 12 and 14 CTAs (the planner's fallback when the power-of-two
+    # clusters of a launch cannot all be resident), odd label counts per CTA
+    # included (their exchange blocks carry a zero pad), on a small random
+    # problem; and the large-label geometry at full K and C on a short sequence
     monkeypatch.setenv("SEMICRF_KERNEL_PATH", "general")
     monkeypatch.setenv("SEMICRF_CL_PLAN", plan)
     if plan.endswith(",0,0"):
-        w = wl.random_small(seed=23, B=3, T=120, K=30, C=56, ragged=True)
-        check_against_oracle(w, run_gpu(w))
-        check_against_oracle(w, run_gpu_fused(w))
-    if not plan.startswith("12"):
+        # 5 labels per CTA with 12 CTAs at C = 56; 4 and 3 with 14 at C = 56 and 41
+        for C in {"12,0,0": (56,), "14,0,0": (56, 41)}[plan]:
+            w = wl.random_small(seed=23, B=3, T=120, K=30, C=C, ragged=True)
+            check_against_oracle(w, run_gpu(w))
+            check_against_oracle(w, run_gpu_fused(w))
+    else:
         w = wl.make_workload("large", B=1, T=700)
         check_against_oracle(w, run_gpu_fused(w))
-        if plan == "14,8,16":
-            check_against_oracle(w, run_gpu(w))
+        check_against_oracle(w, run_gpu(w))
 
 
 def test_kernel_families_agree():
