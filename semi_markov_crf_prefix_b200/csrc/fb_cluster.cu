@@ -643,12 +643,18 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
     }
     // The exchange: each CTA's block of values (its labels, padded with zeros to an
     // even count CgE, so 16-byte units) goes to every CTA of the cluster by one bulk
-    // copy per destination, issued by lane k of warp 0 for CTA k, into position
-    // rank*CgE of the destination's exchange buffer, completing on its mbarrier.
+    // copy per destination, into position rank*CgE of the destination's exchange
+    // buffer, completing on its mbarrier.
     const int CgE = (int)even_up(Cg);
-    const bool issuer = CLUSTER && warp == 0 && lane < g.G;
-    const uint32_t bdst = issuer ? mapa_rank(smem_addr(&sm.gath[rank * CgE]), (uint32_t)lane) : 0u;
-    const uint32_t bbar = issuer ? mapa_rank(smem_addr(&sm.full[0]), (uint32_t)lane) : 0u;
+    // The copies are issued from up to four warps (the owner warps first, then
+    // transition warps), one per scheduler: issuing to many CTAs from one warp
+    // serialises (~70 cycles per destination, measured); warp w lane l sends to
+    // CTA w + nwi*l.
+    const int nwi = g.NWO + g.NWT < 4 ? g.NWO + g.NWT : 4;
+    const int dst_rank = warp + nwi * lane;
+    const bool issuer = CLUSTER && warp < nwi && dst_rank < g.G;
+    const uint32_t bdst = issuer ? mapa_rank(smem_addr(&sm.gath[rank * CgE]), (uint32_t)dst_rank) : 0u;
+    const uint32_t bbar = issuer ? mapa_rank(smem_addr(&sm.full[0]), (uint32_t)dst_rank) : 0u;
     double(&E)[CPL] = *reinterpret_cast<double(*)[CPL]>(&R[0]);
     double &W0 = R[0], &W1 = R[1], &U1 = R[2], &U2 = R[3], &pre = R[4], &f = R[5], &pe = R[6], &w0e = R[7],
            &ap = R[8];
@@ -713,8 +719,7 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
                 // bulk copy per destination CTA
                 if (own) sm.stage[par * CgE + lc] = ap;
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                if (g.NWO > 1) cta_barrier(7, 32 * g.NWO);
-                else __syncwarp();
+                cta_barrier(5, NOT);   // the stage is written, for the issuing warps
                 if (issuer)
                     bulk_to_peer(bdst + par * g.GP * 8, smem_addr(sm.stage + par * CgE), (uint32_t)(CgE * 8),
                                  bbar + par * 8);
@@ -735,9 +740,9 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
                 sm.hbuf[par * Cg + lc] = h;
                 h2 = h1;
                 h1 = h;
-                // prepare position t+1 (row t-1 = U1 is its d = 2 row)
-                prefetch(t + kPF - 1);     // into the slot position t-1 used
-                cp_async_wait<kPF - 2>();  // position t+1 has landed
+                // prepare position t+1 (row t-1 = U1 is its d = 2 row); this step's
+                // prefetch is issued after the new row, off the owners' path to it
+                cp_async_wait<kPF - 3>();  // position t+1 has landed
                 if (t < t_end) prepare(t + 1, u + 1, U1, pre, f_n, pe, w0e, kt_n);
             }
             if constexpr (!CLUSTER) {
@@ -766,10 +771,15 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
                 if (ROWS && c == 0) a.eA[rowbase + t] = kt - kZ;
                 f = f_n;
                 kt = kt_n;
+                prefetch(t + kPF - 1);   // into the slot position t-1 used
             }
         } else if (ro.is_tr) {
             // -------------------------------------------------------- transition
             if constexpr (CLUSTER) {
+                cta_barrier(5, NOT);   // the owners' stage is written
+                if (issuer)
+                    bulk_to_peer(bdst + par * g.GP * 8, smem_addr(sm.stage + par * CgE), (uint32_t)(CgE * 8),
+                                 bbar + par * 8);
                 if (!wait_values<CLUSTER>(sm, par, u, timed_out)) {
                     timed_out = true;
                     set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
@@ -929,12 +939,18 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
     }
     // The exchange: each CTA's block of values (its labels, padded with zeros to an
     // even count CgE, so 16-byte units) goes to every CTA of the cluster by one bulk
-    // copy per destination, issued by lane k of warp 0 for CTA k, into position
-    // rank*CgE of the destination's exchange buffer, completing on its mbarrier.
+    // copy per destination, into position rank*CgE of the destination's exchange
+    // buffer, completing on its mbarrier.
     const int CgE = (int)even_up(Cg);
-    const bool issuer = CLUSTER && warp == 0 && lane < g.G;
-    const uint32_t bdst = issuer ? mapa_rank(smem_addr(&sm.gath[rank * CgE]), (uint32_t)lane) : 0u;
-    const uint32_t bbar = issuer ? mapa_rank(smem_addr(&sm.full[0]), (uint32_t)lane) : 0u;
+    // The copies are issued from up to four warps (the owner warps first, then
+    // transition warps), one per scheduler: issuing to many CTAs from one warp
+    // serialises (~70 cycles per destination, measured); warp w lane l sends to
+    // CTA w + nwi*l.
+    const int nwi = g.NWO + g.NWT < 4 ? g.NWO + g.NWT : 4;
+    const int dst_rank = warp + nwi * lane;
+    const bool issuer = CLUSTER && warp < nwi && dst_rank < g.G;
+    const uint32_t bdst = issuer ? mapa_rank(smem_addr(&sm.gath[rank * CgE]), (uint32_t)dst_rank) : 0u;
+    const uint32_t bbar = issuer ? mapa_rank(smem_addr(&sm.full[0]), (uint32_t)dst_rank) : 0u;
     double(&Er)[CPL] = *reinterpret_cast<double(*)[CPL]>(&R[0]);
     double &W0 = R[0], &W1 = R[1], &V1 = R[2], &V2 = R[3], &pre = R[4], &gg = R[5], &pbe = R[6], &w0e = R[7],
            &coef = R[8], &a2 = R[9], &mu_acc = R[10], &musum = R[11], &bp = R[12], &start = R[13];
@@ -1005,8 +1021,7 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
             if constexpr (CLUSTER) {
                 if (own) sm.stage[par * CgE + lc] = bp;   // as in the forward
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                if (g.NWO > 1) cta_barrier(7, 32 * g.NWO);
-                else __syncwarp();
+                cta_barrier(5, NOT);
                 if (issuer)
                     bulk_to_peer(bdst + par * g.GP * 8, smem_addr(sm.stage + par * CgE), (uint32_t)(CgE * 8),
                                  bbar + par * 8);
@@ -1027,8 +1042,7 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
                 sm.hbuf[par * Cg + lc] = h;
                 h2 = h1;
                 h1 = h;
-                prefetch(s - (kPF - 1));    // into the slot position s+1 used
-                cp_async_wait<kPF - 2>();   // position s-1 has landed
+                cp_async_wait<kPF - 3>();   // position s-1 has landed (the prefetch follows the new row)
                 if (s >= 1) prepare(s - 1, u + 1, V1, pre, gg_n, pbe, w0e, coef_n, a2_n, kb_n);
             }
             if constexpr (!CLUSTER) {
@@ -1066,10 +1080,15 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
                 coef = coef_n;
                 a2 = a2_n;
                 kb = kb_n;
+                prefetch(s - (kPF - 1));   // into the slot position s+1 used
             }
         } else if (ro.is_tr) {
             // ------------------------------------------- transposed transition
             if constexpr (CLUSTER) {
+                cta_barrier(5, NOT);   // the owners' stage is written
+                if (issuer)
+                    bulk_to_peer(bdst + par * g.GP * 8, smem_addr(sm.stage + par * CgE), (uint32_t)(CgE * 8),
+                                 bbar + par * 8);
                 if (!wait_values<CLUSTER>(sm, par, u, timed_out)) {
                     timed_out = true;
                     set_status(a.status, SEMICRF_ERR_DEVICE_TIMEOUT);
