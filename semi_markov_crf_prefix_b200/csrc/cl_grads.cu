@@ -17,7 +17,8 @@
 // term is one FMA, and falls back to exact per-term scaling for the whole CTA
 // only when a pre-scaled row would leave the safe range.
 //
-// Layout: each CTA owns a 32 x 32 tile of outputs ((d, c) or (c, c2)) and a
+// Layout: each CTA owns a tile of outputs (128 or 32 durations x 32 labels for dD,
+// 32 x 32 (c, c2) for dA) and a
 // split z of the (sequence, 32-position chunk) list, which it walks chunk by
 // chunk, staging the chunk's rows in shared memory; it writes its tile of
 // partial sums to part*[z].  A last kernel adds the splits in order (the
@@ -39,20 +40,39 @@ constexpr int kTile = 32;  // output tile edge
 // factor underflowed the product is below 2^-122 (negligible).
 __device__ __forceinline__ bool too_large(double v) { return !(fabs(v) <= 0x1p900); }
 
+// Shared memory of dur_grad_kernel<TD>: X [kCh][kTile] f64 and its references
+// (int), Y [kCh + TD][kTile] f64 and its references.
+template <int TD>
+constexpr size_t dur_smem_bytes()
+{
+    return (size_t)kCh * kTile * 12 + (size_t)(kCh + TD) * kTile * 12;
+}
+
+// TD durations per CTA tile (32 or 128): every staged chunk of rows serves TD
+// durations, so the wider tile stages a quarter as many rows per product.  Warp
+// dq owns the NA = TD/8 consecutive durations d0 + dq NA + k; for start s its
+// lanes need the end rows s + d0 + dq NA + k, a window that slides by one row
+// per start, so each start costs two shared loads (X and the window's new row)
+// for NA FMAs.
+template <int TD>
 __global__ void __launch_bounds__(256) dur_grad_kernel(FbArgs a)
 {
-    __shared__ double xs[kCh][kTile];
-    __shared__ int rs[kCh][kTile];
-    __shared__ double ys[kCh + kTile][kTile];
-    __shared__ int ry[kCh + kTile][kTile];
+    constexpr int NA = TD / 8;   // durations per thread
+    extern __shared__ __align__(16) unsigned char dsm[];
+    double(*xs)[kTile] = reinterpret_cast<double(*)[kTile]>(dsm);
+    double(*ys)[kTile] = reinterpret_cast<double(*)[kTile]>(dsm + (size_t)kCh * kTile * 8);
+    int(*rs)[kTile] = reinterpret_cast<int(*)[kTile]>(dsm + (size_t)(2 * kCh + TD) * kTile * 8);
+    int(*ry)[kTile] = reinterpret_cast<int(*)[kTile]>(dsm + (size_t)(2 * kCh + TD) * kTile * 8 + (size_t)kCh * kTile * 4);
     const int K = a.K, C = a.C, T = a.T;
-    const int z = blockIdx.x, c0 = blockIdx.y * kTile, d0 = 1 + blockIdx.z * kTile;   // d is 1-based
+    const int z = blockIdx.x, c0 = blockIdx.y * kTile, d0 = 1 + blockIdx.z * TD;   // d is 1-based
     const int tid = threadIdx.x, lc = tid & 31, dq = tid >> 5;
     const int c = c0 + lc;
     const bool c_ok = c < C;
     const int nch = (T + kCh - 1) / kCh;
     const long long Q = (long long)a.B * nch;
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    double acc[NA];
+#pragma unroll
+    for (int k = 0; k < NA; ++k) acc[k] = 0.0;
     for (long long q = z; q < Q; q += a.nsD) {
         const int b = (int)(q / nch), s0 = (int)(q % nch) * kCh;
         const int L = a.lengths[b];
@@ -85,7 +105,7 @@ __global__ void __launch_bounds__(256) dur_grad_kernel(FbArgs a)
                 xs[si][l2] = x;
                 rs[si][l2] = r;
             }
-            for (int i = tid; i < (kCh + kTile) * kTile; i += 256) {
+            for (int i = tid; i < (kCh + TD) * kTile; i += 256) {
                 const int ti = i / kTile, l2 = i % kTile, t = s0 + d0 + ti, cc = c0 + l2;
                 double y = 0.0;
                 int r = INT_MIN;
@@ -111,11 +131,17 @@ __global__ void __launch_bounds__(256) dur_grad_kernel(FbArgs a)
             __syncthreads();
         }
         if (!exact) {
-#pragma unroll 4
+            // w[(si + k) % NA] holds end row si + dq NA + k (relative to s0 + d0)
+            double w[NA];
+#pragma unroll
+            for (int k = 0; k < NA; ++k) w[k] = ys[dq * NA + k][lc];
+#pragma unroll
             for (int si = 0; si < kCh; ++si) {
                 const double x = xs[si][lc];
+                const double nxt = ys[si + dq * NA + NA][lc];   // row <= kCh - 1 + TD: staged
 #pragma unroll
-                for (int k = 0; k < 4; ++k) acc[k] = fma(x, ys[si + dq + 8 * k][lc], acc[k]);
+                for (int k = 0; k < NA; ++k) acc[k] = fma(x, w[(si + k) % NA], acc[k]);
+                w[si % NA] = nxt;
             }
         } else {
             for (int si = 0; si < kCh; ++si) {
@@ -123,8 +149,8 @@ __global__ void __launch_bounds__(256) dur_grad_kernel(FbArgs a)
                 const int r = rs[si][lc];
                 if (r == INT_MIN) continue;
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int ti = si + dq + 8 * k;
+                for (int k = 0; k < NA; ++k) {
+                    const int ti = si + dq * NA + k;
                     const double y = ys[ti][lc];
                     if (y != 0.0) acc[k] += scale2c(x * y, ry[ti][lc] - r);
                 }
@@ -132,22 +158,32 @@ __global__ void __launch_bounds__(256) dur_grad_kernel(FbArgs a)
         }
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int d = d0 + dq + 8 * k;
+    for (int k = 0; k < NA; ++k) {
+        const int d = d0 + dq * NA + k;
         if (d <= K && c_ok) a.partD[((size_t)z * K + (d - 1)) * C + c] = acc[k];
     }
 }
 
+// TA x TA outputs (c, c2) per CTA (32 or 64): thread (ti, tj) = (tid / 16,
+// tid % 16) owns the RA x RA outputs c = c0 + RA ti + r, c2 = e0 + tj + 16 k,
+// so a start row costs 2 RA shared loads (the c values as one or two 16-byte
+// loads, the c2 values conflict-free) for RA^2 FMAs.
+template <int TA>
 __global__ void __launch_bounds__(256) trans_grad_kernel(FbArgs a)
 {
-    __shared__ double as[kCh][kTile];
-    __shared__ double bs[kCh][kTile];
+    constexpr int RA = TA / 16;
+    __shared__ __align__(16) double as[kCh][TA];
+    __shared__ double bs[kCh][TA];
     const int C = a.C, T = a.T;
-    const int z = blockIdx.x, c0 = blockIdx.y * kTile, e0 = blockIdx.z * kTile;
-    const int tid = threadIdx.x, ci = tid >> 3, cj = tid & 7;
+    const int z = blockIdx.x, c0 = blockIdx.y * TA, e0 = blockIdx.z * TA;
+    const int tid = threadIdx.x, ti = tid >> 4, tj = tid & 15;
     const int nch = (T + kCh - 1) / kCh;
     const long long Q = (long long)a.B * nch;
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    double acc[RA][RA];
+#pragma unroll
+    for (int r = 0; r < RA; ++r)
+#pragma unroll
+        for (int k = 0; k < RA; ++k) acc[r][k] = 0.0;
     for (long long q = z; q < Q; q += a.nsA) {
         const int b = (int)(q / nch), s0 = (int)(q % nch) * kCh;
         const int L = a.lengths[b];
@@ -155,8 +191,8 @@ __global__ void __launch_bounds__(256) trans_grad_kernel(FbArgs a)
         const size_t rowbase = (size_t)b * (T + 1);
         const double g = a.grad ? a.grad[b] : 1.0;
         __syncthreads();
-        for (int i = tid; i < kCh * kTile; i += 256) {
-            const int si = i / kTile, l2 = i % kTile, s = s0 + si;
+        for (int i = tid; i < kCh * TA; i += 256) {
+            const int si = i / TA, l2 = i % TA, s = s0 + si;
             const bool ok = s >= 1 && s <= L - 1;
             double x = 0.0, y = 0.0;
             if (ok && c0 + l2 < C) {
@@ -170,16 +206,29 @@ __global__ void __launch_bounds__(256) trans_grad_kernel(FbArgs a)
         __syncthreads();
 #pragma unroll 4
         for (int si = 0; si < kCh; ++si) {
-            const double x = as[si][ci];
+            double x[RA], y[RA];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) acc[k] = fma(x, bs[si][cj + 8 * k], acc[k]);
+            for (int r = 0; r < RA; r += 2) {
+                const double2 v = *reinterpret_cast<const double2 *>(&as[si][RA * ti + r]);
+                x[r] = v.x;
+                x[r + 1] = v.y;
+            }
+#pragma unroll
+            for (int k = 0; k < RA; ++k) y[k] = bs[si][tj + 16 * k];
+#pragma unroll
+            for (int r = 0; r < RA; ++r)
+#pragma unroll
+                for (int k = 0; k < RA; ++k) acc[r][k] = fma(x[r], y[k], acc[r][k]);
         }
     }
-    const int c = c0 + ci;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int e = e0 + cj + 8 * k;
-        if (c < C && e < C) a.partA[((size_t)z * C + c) * C + e] = acc[k];
+    for (int r = 0; r < RA; ++r) {
+        const int c = c0 + RA * ti + r;
+#pragma unroll
+        for (int k = 0; k < RA; ++k) {
+            const int e = e0 + tj + 16 * k;
+            if (c < C && e < C) a.partA[((size_t)z * C + c) * C + e] = acc[r][k];
+        }
     }
 }
 
@@ -325,14 +374,58 @@ __global__ void cov_musum_kernel(FbArgs a)
 
 }  // namespace
 
-// Splits so that each contraction launches about four CTAs per SM.
+// Duration tile of the dD contraction: 128 durations per CTA when K reaches it.
+inline int dur_tile(int K) { return K >= 128 ? 128 : kTile; }
+
+// Resident CTAs per SM of the dD contraction (the runtime's figure; without a
+// device, the one its register and shared-memory use gives on sm_100a).
+int dur_grad_occupancy(int TD)
+{
+    int n = 0;
+    cudaError_t e;
+    if (TD == 128) {
+        e = cudaFuncSetAttribute(dur_grad_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)dur_smem_bytes<128>());
+        if (e == cudaSuccess)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dur_grad_kernel<128>, 256, dur_smem_bytes<128>());
+    } else {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dur_grad_kernel<kTile>, 256, dur_smem_bytes<kTile>());
+    }
+    if (e != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = TD == 128 ? 3 : 5;
+    }
+    return n;
+}
+
+// Output tile of the dA contraction: 64 x 64 when C exceeds 32.
+inline int trans_tile(int C) { return C > kTile ? 64 : kTile; }
+
+int trans_grad_occupancy(int TA)
+{
+    int n = 0;
+    const cudaError_t e = TA == 64 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, trans_grad_kernel<64>, 256, 0)
+                                   : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, trans_grad_kernel<kTile>, 256, 0);
+    if (e != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = TA == 64 ? 3 : 4;
+    }
+    return n;
+}
+
+// Splits: each contraction fills two waves of resident CTAs (every CTA walks the
+// same number of chunks, so a partial last wave would idle the rest).
 void cl_grad_splits(int B, int T, int K, int C, int *nsD, int *nsA)
 {
     const long long Q = (long long)B * ceil_div(T, kCh);
-    const int tilesD = ceil_div(K, kTile) * ceil_div(C, kTile);
-    const int tilesA = ceil_div(C, kTile) * ceil_div(C, kTile);
+    const int tilesD = ceil_div(K, dur_tile(K)) * ceil_div(C, kTile);
+    const int tilesA = ceil_div(C, trans_tile(C)) * ceil_div(C, trans_tile(C));
     const int nsm = device_sm_count();
-    long long d = ceil_div(4 * nsm, tilesD), e = ceil_div(4 * nsm, tilesA);
+    const long long slotsD = 2LL * nsm * dur_grad_occupancy(dur_tile(K));
+    const long long slotsA = 2LL * nsm * trans_grad_occupancy(trans_tile(C));
+    long long d = slotsD / tilesD, e = slotsA / tilesA;
+    if (d < 1) d = 1;
+    if (e < 1) e = 1;
     if (d > 1024) d = 1024;
     if (e > 1024) e = 1024;
     *nsD = (int)(d < Q ? d : Q);
@@ -374,11 +467,26 @@ cudaError_t launch_coverage(const FbArgs &a, cudaStream_t st)
 
 cudaError_t launch_cl_param_grads(const FbArgs &a, cudaStream_t st)
 {
+    if (dur_tile(a.K) == 128) {
+        const size_t smem = dur_smem_bytes<128>();
+        cudaError_t e = cudaFuncSetAttribute(dur_grad_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        prof_before(st);
+        dur_grad_kernel<128><<<dim3(a.nsD, ceil_div(a.C, kTile), ceil_div(a.K, 128)), 256, smem, st>>>(a);
+        prof_after(st);
+    } else {
+        prof_before(st);
+        dur_grad_kernel<kTile><<<dim3(a.nsD, ceil_div(a.C, kTile), ceil_div(a.K, kTile)), 256, dur_smem_bytes<kTile>(),
+                                 st>>>(a);
+        prof_after(st);
+    }
     prof_before(st);
-    dur_grad_kernel<<<dim3(a.nsD, ceil_div(a.C, kTile), ceil_div(a.K, kTile)), 256, 0, st>>>(a);
-    prof_after(st);
-    prof_before(st);
-    trans_grad_kernel<<<dim3(a.nsA, ceil_div(a.C, kTile), ceil_div(a.C, kTile)), 256, 0, st>>>(a);
+    const int TA = trans_tile(a.C);
+    if (TA == 64)
+        trans_grad_kernel<64><<<dim3(a.nsA, ceil_div(a.C, 64), ceil_div(a.C, 64)), 256, 0, st>>>(a);
+    else
+        trans_grad_kernel<kTile><<<dim3(a.nsA, ceil_div(a.C, kTile), ceil_div(a.C, kTile)), 256, 0, st>>>(a);
     prof_after(st);
     const int n = a.C * a.C + a.K * a.C;   // one warp per output
     int blocks = ceil_div((long long)n * 32, 256);

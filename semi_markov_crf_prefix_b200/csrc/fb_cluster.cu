@@ -64,6 +64,12 @@ namespace semicrf {
 namespace {
 
 constexpr int kPF = 8;                        // exp-table prefetch ring depth (positions)
+// Named barriers between the owner and the window warps, two each so that
+// consecutive steps alternate: kBarRow + (u & 1) the owners' new row of step u
+// (owners arrive, window warps wait), kBarWin + (u & 1) the window sums of step u
+// (window warps arrive, owners wait).  Ids 1-5 and 7 serve the other roles.
+constexpr int kBarRow = 8;
+constexpr int kBarWin = 10;
 constexpr long long kWaitCycles = 1ll << 31;  // ~1 s at 2 GHz
 
 __device__ __forceinline__ void cta_barrier(int id, int nthreads)
@@ -74,21 +80,6 @@ __device__ __forceinline__ void cta_barrier(int id, int nthreads)
 __device__ __forceinline__ void cta_arrive(int id, int nthreads)
 {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// bar.sync with an OR over the threads' flags: every thread gets the same answer
-__device__ __forceinline__ bool cta_barrier_or(int id, int nthreads, bool v)
-{
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)v), "r"(id), "r"(nthreads)
-        : "memory");
-    return r != 0;
 }
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
@@ -201,7 +192,7 @@ struct ClSmem {
     double *pf_es, *pf_ies, *pf_cu, *pf_ca;   // [kPF][Cg] prefetch rings
     uint64_t *full;  // [2] exchange mbarriers
     int *pf_m, *pf_eu, *pf_ea;                // [kPF][Cg] each
-    int *hbuf;       // [2][Cg] rebase exponent of each label at the last two positions
+    int *hbuf;       // [4][Cg] rebase exponent of each label at the last four positions
     int *kbuf;       // [4]     normaliser exponents
 };
 
@@ -219,7 +210,7 @@ __host__ __device__ __forceinline__ size_t cl_smem_bytes_impl(int K, int C, cons
     const size_t npf = bwd ? 4 : 2;
     const size_t nd = cl_head_doubles(K, g) + 2 * (size_t)g.GP + 2 * even_up(g.Cg) + even_up(g.Cg) +
                       4 * (size_t)g.Cg * g.PW + npf * kPF * g.Cg;
-    const size_t ni = (bwd ? 3 : 1) * (size_t)kPF * g.Cg + 2 * (size_t)g.Cg + 4;
+    const size_t ni = (bwd ? 3 : 1) * (size_t)kPF * g.Cg + 4 * (size_t)g.Cg + 4;
     return nd * sizeof(double) + 2 * sizeof(uint64_t) + ni * sizeof(int);
 }
 
@@ -242,7 +233,7 @@ __device__ __forceinline__ ClSmem cl_smem(double *base, int K, int C, const ClGe
     s.pf_eu = s.pf_m + kPF * g.Cg;
     s.pf_ea = bwd ? s.pf_eu + kPF * g.Cg : s.pf_eu;
     s.hbuf = bwd ? s.pf_ea + kPF * g.Cg : s.pf_eu;
-    s.kbuf = s.hbuf + 2 * g.Cg;
+    s.kbuf = s.hbuf + 4 * g.Cg;
     return s;
 }
 
@@ -521,7 +512,7 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
     extern __shared__ __align__(16) double smc[];
     const int K = a.K, C = a.C, Cg = g.Cg, NT = g.NT, RS = g.RS, PW = g.PW;
     const int NOT = 32 * (g.NWO + g.NWT);   // owner + transition threads
-    const int W0T = 32 * (g.NWO + g.NWT);   // first window thread
+    const int NOW = 32 * (g.NWO + g.NWW);   // owner + window threads
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rank = CLUSTER ? (int)cluster_rank() : 0;
     int b, seg;
@@ -580,7 +571,7 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
         for (int i = tid; i < 2 * g.GP; i += NT) sm.gath[i] = 0.0;
         for (int i = tid; i < 2 * (int)even_up(Cg); i += NT) sm.stage[i] = 0.0;
         for (int i = tid; i < 4 * Cg * PW; i += NT) sm.pre3[i] = 0.0;
-        for (int i = tid; i < 2 * Cg; i += NT) sm.hbuf[i] = 0;
+        for (int i = tid; i < 4 * Cg; i += NT) sm.hbuf[i] = 0;
         if (tid == 0) {
             if constexpr (RECOMPUTE) {
                 const int32_t *ck_r = reinterpret_cast<const int32_t *>(ck_ring + (size_t)K * C);
@@ -737,9 +728,12 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
                     f *= s2;
                     U1 *= s2;
                 }
-                sm.hbuf[par * Cg + lc] = h;
+                sm.hbuf[(u & 3) * Cg + lc] = h;
                 h2 = h1;
                 h1 = h;
+            }
+            if (u >= 1 && t < t_end) cta_barrier(kBarWin + ((u - 1) & 1), NOW);   // window sums of step u-1
+            if (own) {
                 // prepare position t+1 (row t-1 = U1 is its d = 2 row); this step's
                 // prefetch is issued after the new row, off the owners' path to it
                 cp_async_wait<kPF - 3>();  // position t+1 has landed
@@ -773,9 +767,13 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
                 kt = kt_n;
                 prefetch(t + kPF - 1);   // into the slot position t-1 used
             }
+            if (t < t_end) cta_arrive(kBarRow + (u & 1), NOW);   // row t and h_t stored, for the window
         } else if (ro.is_tr) {
             // -------------------------------------------------------- transition
             if constexpr (CLUSTER) {
+                // this position's exchange: every CTA's block, G*CgE doubles (the
+                // barrier's phase for position t-2 completed at this warp's last wait)
+                if (tid == 32 * g.NWO) mbar_expect_tx(&sm.full[par], g.G * (int)even_up(Cg) * 8);
                 cta_barrier(5, NOT);   // the owners' stage is written
                 if (issuer)
                     bulk_to_peer(bdst + par * g.GP * 8, smem_addr(sm.stage + par * CgE), (uint32_t)(CgE * 8),
@@ -812,8 +810,10 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
             }
         } else if (ro.is_win) {
             // ------------------------------------- window sums two positions ahead
-            if (CLUSTER && tid == W0T) mbar_expect_tx(&sm.full[par], g.G * (int)even_up(Cg) * 8);
-            const int hp = ro.lab_ok ? sm.hbuf[(par ^ 1) * Cg + lc] : 0;   // rebase at t-1
+            // They run a position ahead of the owners at most: row t-1 and h_{t-1}
+            // come from the owners' step u-1, the sums go to their step u+1.
+            if (u >= 1) cta_barrier(kBarRow + ((u - 1) & 1), NOW);
+            const int hp = ro.lab_ok ? sm.hbuf[((u - 1) & 3) * Cg + lc] : 0;   // rebase at t-1
             const int tau2K = tK + 2 >= K ? tK + 2 - K : tK + 2;   // K >= 3 whenever a row is read
             double v = 0.0;
             if (ro.lab_ok)
@@ -821,9 +821,10 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
                          : window_fwd(sm.ring, sm.Wd, K, RS, lc, g.LPW, j, tau2K, hp);
             const double s = group_sum(v, g.LPW < 32 ? g.LPW : 32);
             if (ro.lab_ok && (j & 31) == 0) sm.pre3[((u + 2) & 3) * Cg * PW + lc * PW + (j >> 5)] = s;
+            if (t + 1 < t_end) cta_arrive(kBarWin + (u & 1), NOW);
         }
-        if (cta_barrier_or(2, NT, timed_out)) timed_out = true;
         if (CKPT && td == 0 && t < L) {
+            cta_barrier(2, NT);   // every role is through step u
             // checkpoint t / delta: the ring at the reference of position t, r, k_{t+1}, k_{t+2}.
             // Row age 0 (row t) is there; ages 1..K-2 are at the reference of t-1; the
             // oldest row (age K-1, K >= 3) at that of t-2.
@@ -836,8 +837,8 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
                     int age = tK - sl;
                     if (age < 0) age += K;
                     int hh = 0;
-                    if (age >= 1) hh = sm.hbuf[par * Cg + l2];
-                    if (age == K - 1 && K >= 3) hh += sm.hbuf[(par ^ 1) * Cg + l2];
+                    if (age >= 1) hh = sm.hbuf[(u & 3) * Cg + l2];
+                    if (age == K - 1 && K >= 3) hh += sm.hbuf[((u - 1) & 3) * Cg + l2];
                     ck_ring[(size_t)sl * C + c0l + l2] = rescale(sm.ring[sl * RS + l2], hh);
                 }
             }
@@ -870,7 +871,7 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
     extern __shared__ __align__(16) double smc[];
     const int K = a.K, C = a.C, Cg = g.Cg, NT = g.NT, RS = g.RS, PW = g.PW;
     const int NOT = 32 * (g.NWO + g.NWT);
-    const int W0T = 32 * (g.NWO + g.NWT);
+    const int NOW = 32 * (g.NWO + g.NWW);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rank = CLUSTER ? (int)cluster_rank() : 0;
     const int L = a.lengths[b];
@@ -905,7 +906,7 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
     for (int i = tid; i < 2 * g.GP; i += NT) sm.gath[i] = 0.0;
     for (int i = tid; i < 2 * (int)even_up(Cg); i += NT) sm.stage[i] = 0.0;
     for (int i = tid; i < 4 * Cg * PW; i += NT) sm.pre3[i] = 0.0;   // positions L-1, L-2: no rows beyond L
-    for (int i = tid; i < 2 * Cg; i += NT) sm.hbuf[i] = 0;
+    for (int i = tid; i < 4 * Cg; i += NT) sm.hbuf[i] = 0;
     if (tid == 0) {
         sm.kbuf[0] = 0;
         sm.kbuf[1] = 0;
@@ -1039,9 +1040,12 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
                     gg *= s2;
                     V1 *= s2;
                 }
-                sm.hbuf[par * Cg + lc] = h;
+                sm.hbuf[(u & 3) * Cg + lc] = h;
                 h2 = h1;
                 h1 = h;
+            }
+            if (u >= 1 && s >= 1) cta_barrier(kBarWin + ((u - 1) & 1), NOW);   // window sums of step u-1
+            if (own) {
                 cp_async_wait<kPF - 3>();   // position s-1 has landed (the prefetch follows the new row)
                 if (s >= 1) prepare(s - 1, u + 1, V1, pre, gg_n, pbe, w0e, coef_n, a2_n, kb_n);
             }
@@ -1082,9 +1086,11 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
                 kb = kb_n;
                 prefetch(s - (kPF - 1));   // into the slot position s+1 used
             }
+            if (s >= 1) cta_arrive(kBarRow + (u & 1), NOW);   // row s and h_s stored, for the window
         } else if (ro.is_tr) {
             // ------------------------------------------- transposed transition
             if constexpr (CLUSTER) {
+                if (tid == 32 * g.NWO) mbar_expect_tx(&sm.full[par], g.G * (int)even_up(Cg) * 8);   // as forward
                 cta_barrier(5, NOT);   // the owners' stage is written
                 if (issuer)
                     bulk_to_peer(bdst + par * g.GP * 8, smem_addr(sm.stage + par * CgE), (uint32_t)(CgE * 8),
@@ -1113,16 +1119,16 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
             }
         } else if (ro.is_win) {
             // ----------------------- window sums two positions ahead (position s-2)
-            if (CLUSTER && tid == W0T) mbar_expect_tx(&sm.full[par], g.G * (int)even_up(Cg) * 8);
-            const int hp = ro.lab_ok ? sm.hbuf[(par ^ 1) * Cg + lc] : 0;   // rebase at s+1
+            if (u >= 1) cta_barrier(kBarRow + ((u - 1) & 1), NOW);   // row s+1, h_{s+1} (as forward)
+            const int hp = ro.lab_ok ? sm.hbuf[((u - 1) & 3) * Cg + lc] : 0;   // rebase at s+1
             double v = 0.0;
             if (ro.lab_ok)
                 v = wreg ? window_bwd_nr<NU>(g.NRB, sm.ring, K, RS, lc, g.LPW, j, sK, hp, R)
                          : window_bwd(sm.ring, sm.Wd, K, RS, lc, g.LPW, j, sK, hp);
             const double sum = group_sum(v, g.LPW < 32 ? g.LPW : 32);
             if (ro.lab_ok && (j & 31) == 0 && s >= 2) sm.pre3[((u + 2) & 3) * Cg * PW + lc * PW + (j >> 5)] = sum;
+            if (s >= 2) cta_arrive(kBarWin + (u & 1), NOW);
         }
-        if (cta_barrier_or(2, NT, timed_out)) timed_out = true;
         sK = (sK == 0) ? K - 1 : sK - 1;
     }
     if (own) {

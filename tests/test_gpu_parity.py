@@ -380,14 +380,15 @@ def test_fused_random_shapes(seed, B, T, K, C):
     check_against_oracle(w, run_gpu_fused(w))
 
 
-@pytest.mark.parametrize("path", [None, "general"])
-def test_fused_rebased_columns(path, monkeypatch):
+@pytest.mark.parametrize("path,K", [(None, 12), ("general", 12), (None, 160)])
+def test_fused_rebased_columns(path, K, monkeypatch):
     # emissions of standard deviation 12: log Z grows by ~18 per position, so the
     # per-label references of both chains move every few dozen positions and the
-    # passes over the stored rows take their exact-scaling branch
+    # passes over the stored rows take their exact-scaling branch (K = 160: the
+    # dD contraction's 128-duration tile)
     if path:
         monkeypatch.setenv("SEMICRF_KERNEL_PATH", path)
-    w = wl.random_small(15, 4, 400, 12, 9, ragged=True, scale=12.0)
+    w = wl.random_small(15, 4, 400, K, 9, ragged=True, scale=12.0)
     grad = np.array([1.0, -0.5, 2.0, 0.25])
     check_against_oracle(w, run_gpu_fused(w, grad=grad), grad=grad)
 
