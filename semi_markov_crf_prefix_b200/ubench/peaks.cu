@@ -111,8 +111,9 @@ int main(int argc, char **argv)
     float *d32;
     CK(cudaMalloc(&d64, sizeof(double)));
     CK(cudaMalloc(&d32, sizeof(float)));
-    // about 60 ms per launch at the nominal rates (64, 128 and 16 per SM per clock)
-    const int it64 = 512, it32 = 2048, itx = 128;
+    // about 5 ms per launch at the nominal rates (64, 128 and 16 per SM per clock),
+    // long against launch and ramp-up costs
+    const int it64 = 32768, it32 = 131072, itx = 8192;
     const double per = (double)blocks * threads * NCH;
     double ms64, ms32, msx;
     if (time_it([&] { k_fp64<<<blocks, threads>>>(d64, 0.999999, 1e-7, it64); }, reps, &ms64)) return 1;
