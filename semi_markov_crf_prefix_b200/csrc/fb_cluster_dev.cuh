@@ -277,14 +277,30 @@ __device__ __forceinline__ double strided_dot(const double *u, int ustep, const 
 }
 
 // The lane's window rows m in [m0, n), at ring slots sl0 + m*dsl (dsl = -LPW in
-// the forward, +LPW in the backward), times the exact power of two 2^h in both
-// copies (scale2c's two factors).  Row by row and not unrolled (the loads and
-// stores alias, so unrolling overlaps nothing and costs registers the rest of the
-// kernel needs); staging several loads ahead measured slower on the large-label
-// chains.
+// the forward, +LPW in the backward), times the power of two 2^h in both copies:
+// one multiplication when 2^h is a normal double, else scale2c's two factors
+// (either way exact unless the result leaves the normal range).  This runs on
+// the rebase positions that set the chain's pace, and each row's store waits on
+// its multiply: dropping the second multiply cut the large-label step by 4 %.
+// Row by row and not unrolled (the loads and stores alias, so unrolling
+// overlaps nothing and costs registers the rest of the kernel needs); staging
+// rows ahead, a software-pipelined loop and an exponent-field add all measured
+// slower on the large-label chains.
 __device__ __forceinline__ void rescale_rows(double *ring, int K, int RS, int lc, int sl0, int dsl, int m0, int n,
                                              int h)
 {
+    if (h >= -1022 && h <= 1023) {   // 2^h is a normal double
+        const double s = pow2c(h);
+#pragma unroll 1
+        for (int m = m0; m < n; ++m) {
+            const int sl = sl0 + m * dsl;
+            const int other = sl >= K ? sl - K : sl + K;
+            const double w = ring[sl * RS + lc] * s;
+            ring[sl * RS + lc] = w;
+            ring[other * RS + lc] = w;
+        }
+        return;
+    }
     const int h1 = h / 2;
     const double s2a = pow2c(h1), s2b = pow2c(h - h1);
 #pragma unroll 1
@@ -344,10 +360,10 @@ __device__ __forceinline__ double window_fwd_reg(double *ring, int K, int RS, in
     if (hp != 0 && d0 <= K) rescale_rows(ring, K, RS, lc, tauK + K - d0, -LPW, d0 < 4 ? 1 : 0, (K - d0) / LPW + 1, hp);
     const double *p = ring + (tauK + K - d0) * RS + lc;
     const int step = LPW * RS;
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-    for (int m = 0; m < NR; ++m) acc[m & 3] = fma(p[-m * step], W[m], acc[m & 3]);
-    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    for (int m = 0; m < NR; ++m) acc[m & 7] = fma(p[-m * step], W[m], acc[m & 7]);
+    return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
 template <int NR, int NU>
@@ -360,10 +376,10 @@ __device__ __forceinline__ double window_bwd_reg(double *ring, int K, int RS, in
         rescale_rows(ring, K, RS, lc, sK + i0, LPW, i0 < 2 ? 1 : 0, (K - 2 - i0) / LPW + 1, hp);
     const double *p = ring + (sK + i0) * RS + lc;
     const int step = LPW * RS;
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-    for (int m = 0; m < NR; ++m) acc[m & 3] = fma(p[m * step], W[m], acc[m & 3]);
-    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    for (int m = 0; m < NR; ++m) acc[m & 7] = fma(p[m * step], W[m], acc[m & 7]);
+    return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
 // Window sum with the row count of the plan's bucket (8, 16 or 32 rows per lane).
