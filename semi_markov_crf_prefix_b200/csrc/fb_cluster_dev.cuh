@@ -70,6 +70,8 @@ constexpr int kBarWin = 10;
 // Cluster kernels: the owners' values for the next exchange are published
 // (owners arrive, transition warps wait), once per step.
 constexpr int kBarPub = 6;
+// The window warps among themselves: rows of rebased labels rescaled (step u).
+constexpr int kBarResc = 12;
 constexpr long long kWaitCycles = 1ll << 31;  // ~1 s at 2 GHz
 
 __device__ __forceinline__ void cta_barrier(int id, int nthreads)
@@ -311,6 +313,43 @@ __device__ __forceinline__ void rescale_rows(double *ring, int K, int RS, int lc
         ring[sl * RS + lc] = w;
         ring[other * RS + lc] = w;
     }
+}
+
+// The stored rows of every label that rebased one position earlier, brought to
+// its new reference by all the window lanes together (wl of nw): n rows per
+// label at ring slots sl0 + i*dsl, both copies, times 2^h as rescale_rows does.
+// A rebase is a few positions' burst over all labels of a chain, and on those
+// positions the slowest CTA sets the cluster's pace: spread over every window
+// lane a label's rows take about two rounds instead of a 32-row loop in its
+// own lanes.  Returns whether any label rebased, the same answer in every
+// window warp (they read the same exponents), so the barrier after it is
+// uniform.
+__device__ __forceinline__ bool coop_rescale(double *ring, const int *hrow, int K, int RS, int cg_own, int sl0,
+                                             int dsl, int n, int wl, int nw, int lane)
+{
+    unsigned any = 0;
+    for (int l0 = 0; l0 < cg_own; l0 += 32) {
+        const int hl = l0 + lane < cg_own ? hrow[l0 + lane] : 0;
+        unsigned mask = __ballot_sync(0xffffffffu, hl != 0);
+        any |= mask;
+        while (mask) {
+            const int bit = __ffs(mask) - 1;
+            mask &= mask - 1;
+            const int h = __shfl_sync(0xffffffffu, hl, bit), l = l0 + bit;
+            const bool one = h >= -1022 && h <= 1023;   // 2^h is a normal double
+            const int h1 = h / 2;
+            const double s = pow2c(h), s2a = pow2c(h1), s2b = pow2c(h - h1);
+            for (int i = wl; i < n; i += nw) {
+                const int sl = sl0 + i * dsl;
+                const int other = sl >= K ? sl - K : sl + K;
+                const double v = ring[sl * RS + l];
+                const double w = one ? v * s : (v * s2a) * s2b;
+                ring[sl * RS + l] = w;
+                ring[other * RS + l] = w;
+            }
+        }
+    }
+    return any != 0;
 }
 
 // Forward window: sum over d = d0 + m*LPW <= K (d0 = 3 + j) of ring row (tau - d)
@@ -848,8 +887,18 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
             // They run a position ahead of the owners at most: row t-1 and h_{t-1}
             // come from the owners' step u-1, the sums go to their step u+1.
             if (u >= 1) cta_barrier(kBarRow + ((u - 1) & 1), NOW);
-            const int hp = ro.lab_ok ? sm.hbuf[((u - 1) & 3) * Cg + lc] : 0;   // rebase at t-1
             const int tau2K = tK + 2 >= K ? tK + 2 - K : tK + 2;   // K >= 3 whenever a row is read
+            // rebases at t-1: rows d = 4..K of those labels (row d = 3 was written after
+            // it), by all window lanes together on TS plans (many labels per CTA, few
+            // lanes each), else by each label's own lanes inside its window sum
+            int hp = ro.lab_ok ? sm.hbuf[((u - 1) & 3) * Cg + lc] : 0;
+            if constexpr (ts) {
+                const int wl = tid - 32 * (g.NWO + g.NWT), nw = 32 * g.NWW;   // window lane index
+                if (coop_rescale(sm.ring, sm.hbuf + ((u - 1) & 3) * Cg, K, RS, cg_own, tau2K + K - 4, -1, K - 3, wl,
+                                 nw, lane))
+                    cta_barrier(kBarResc, nw);
+                hp = 0;   // the rows are at the new reference
+            }
             double v = 0.0;
             if (ro.lab_ok)
                 v = wreg ? window_fwd_nr<NU>(g.NRB, sm.ring, K, RS, lc, g.LPW, j, tau2K, hp, R)
@@ -1188,7 +1237,15 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
         } else if (ro.is_win) {
             // ----------------------- window sums two positions ahead (position s-2)
             if (u >= 1) cta_barrier(kBarRow + ((u - 1) & 1), NOW);   // row s+1, h_{s+1} (as forward)
-            const int hp = ro.lab_ok ? sm.hbuf[((u - 1) & 3) * Cg + lc] : 0;   // rebase at s+1
+            // rebases at s+1: rows i = 2..K-2 of those labels (as forward)
+            int hp = ro.lab_ok ? sm.hbuf[((u - 1) & 3) * Cg + lc] : 0;
+            if constexpr (ts) {
+                const int wl = tid - 32 * (g.NWO + g.NWT), nw = 32 * g.NWW;   // window lane index
+                if (coop_rescale(sm.ring, sm.hbuf + ((u - 1) & 3) * Cg, K, RS, cg_own, sK + 2, 1, K - 3, wl, nw,
+                                 lane))
+                    cta_barrier(kBarResc, nw);
+                hp = 0;
+            }
             double v = 0.0;
             if (ro.lab_ok)
                 v = wreg ? window_bwd_nr<NU>(g.NRB, sm.ring, K, RS, lc, g.LPW, j, sK, hp, R)
