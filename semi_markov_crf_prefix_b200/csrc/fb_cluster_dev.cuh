@@ -10,14 +10,16 @@
 // summary 2.A-2.C).  A CTA has three kinds of warps.  Owner warps run the chain
 // of one label per lane; transition warps form the C x C product; window warps
 // form the duration sums.  The sequential chain of one position is
-//   send:        a'[t,c] = U[t-1] (W0 e) + pre e into a stage buffer; one bulk
-//                copy of the CTA's block of values (cp.async.bulk, shared::cta
-//                to shared::cluster, no multicast) to every CTA of the cluster,
-//                completing its bytes on that CTA's mbarrier for the position
-//                (G = 1: a plain store + bar.arrive).  TS = 0: the owners form
-//                and send it; TS = 1: the transition lanes of the label form it
-//                right after their sum of the previous position, from values the
-//                owners published, and send it;
+//   send:        a'[t,c] = U[t-1] (W0 e) + pre e to every CTA of the cluster,
+//                completing its bytes on that CTA's mbarrier for the position.
+//                TS = 0: the owners form it into a stage buffer and up to four
+//                warps issue one bulk copy of the CTA's block per destination
+//                (cp.async.bulk, shared::cta to shared::cluster, no multicast).
+//                TS = 1: the transition lanes of the label form it right after
+//                their sum of the previous position, from values the owners
+//                published, and lane j stores it into CTAs j, j + LPL, ... with
+//                st.async (no stage, fence or barrier before the send).
+//                G = 1: a plain store + bar.arrive;
 //   transition:  wait on the mbarrier, q[c] = sum_c' a'[t,c'] exp(A[c',c])
 //                (LPL lanes per label, CPL terms each, shuffle reduction);
 //                bar.arrive to the owners; the lanes of the first label also
@@ -159,6 +161,15 @@ __device__ __forceinline__ void bulk_to_peer(uint32_t dst, uint32_t src, uint32_
 {
     asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "r"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// st.async of v to the shared::cluster address ra, completing 8 bytes on the
+// mbarrier at the shared::cluster address rb.
+__device__ __forceinline__ void st_async_at(uint32_t ra, uint32_t rb, double v)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];" ::"r"(ra),
+                 "l"(__double_as_longlong(v)), "r"(rb)
                  : "memory");
 }
 
@@ -680,6 +691,8 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
     const bool issuer = CLUSTER && warp >= iw0 && warp < iw0 + nwi && dst_rank < g.G;
     const uint32_t bdst = issuer ? mapa_rank(smem_addr(&sm.gath[rank * CgE]), (uint32_t)dst_rank) : 0u;
     const uint32_t bbar = issuer ? mapa_rank(smem_addr(&sm.full[0]), (uint32_t)dst_rank) : 0u;
+    // TS: a label's value goes from its own lanes to every CTA by st.async
+    const uint32_t xg = smem_addr(&sm.gath[rank * CgE + (ro.lab_ok ? lc : 0)]), xb = smem_addr(&sm.full[0]);
     double(&E)[CPL] = *reinterpret_cast<double(*)[CPL]>(&R[0]);
     double &W0 = R[0], &W1 = R[1], &U1 = R[2], &U2 = R[3], &pre = R[4], &f = R[5], &pe = R[6], &w0e = R[7],
            &ap = R[8];
@@ -732,10 +745,10 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
     if (ts) {
         // a'[t0+1] from the owners; from then on the transition lanes form each
         // position's value from the previous q and send it
-        if (own) sm.stage[lc] = fma(U1, w0e, pe);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncthreads();
-        if (issuer) bulk_to_peer(bdst, smem_addr(sm.stage), (uint32_t)(CgE * 8), bbar);
+        if (own) {
+            const double a0 = fma(U1, w0e, pe);
+            for (int dr = 0; dr < g.G; ++dr) st_async_at(mapa_rank(xg, dr), mapa_rank(xb, dr), a0);
+        }
     }
 
     int tK = (t0 + 1) % K;
@@ -827,7 +840,7 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
             if constexpr (CLUSTER) {
                 // this position's exchange: every CTA's block, G*CgE doubles (the
                 // barrier's phase for position t-2 completed at this warp's last wait)
-                if (tid == 32 * g.NWO) mbar_expect_tx(&sm.full[par], g.G * (int)even_up(Cg) * 8);
+                if (tid == 32 * g.NWO) mbar_expect_tx(&sm.full[par], ts ? C * 8 : g.G * (int)even_up(Cg) * 8);
                 if (!ts) {
                     cta_barrier(5, NOT);   // the owners' stage is written
                     if (issuer)
@@ -849,16 +862,13 @@ __device__ __forceinline__ void cl_fwd_body(const FbArgs &a, const ClGeom &g, in
             group_sum2(q, n, g.LPL);
             if (ts) {
                 cta_barrier(kBarPub, NOT);   // the owners' values of this step
-                if (t < t_end) {
-                    // a'[t+1], the owners' own FMA one step early, into the stage; then one
-                    // bulk copy per destination CTA
-                    if (ro.lab_ok && j == 0)
-                        sm.stage[(par ^ 1) * CgE + lc] = fma(q * sm.pub[lc], sm.pub[CgE + lc], sm.pub[2 * CgE + lc]);
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    cta_barrier(5, 32 * g.NWT);   // every label's value is staged
-                    if (issuer)
-                        bulk_to_peer(bdst + (par ^ 1) * g.GP * 8, smem_addr(sm.stage + (par ^ 1) * CgE),
-                                     (uint32_t)(CgE * 8), bbar + (par ^ 1) * 8);
+                if (t < t_end && ro.lab_ok) {
+                    // a'[t+1], the owners' own FMA one step early, from every lane of the
+                    // label; lane j stores it into CTAs j, j + LPL, ... (st.async, completing
+                    // 8 bytes on that CTA's mbarrier for the position)
+                    const double an = fma(q * sm.pub[lc], sm.pub[CgE + lc], sm.pub[2 * CgE + lc]);
+                    const uint32_t og = xg + (uint32_t)((par ^ 1) * g.GP * 8), ob = xb + (uint32_t)((par ^ 1) * 8);
+                    for (int dr = j; dr < g.G; dr += g.LPL) st_async_at(mapa_rank(og, dr), mapa_rank(ob, dr), an);
                 }
             }
             if (ro.lab_ok && j == 0) sm.qbuf[par * CgE + lc] = q;
@@ -1038,6 +1048,8 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
     const bool issuer = CLUSTER && warp >= iw0 && warp < iw0 + nwi && dst_rank < g.G;
     const uint32_t bdst = issuer ? mapa_rank(smem_addr(&sm.gath[rank * CgE]), (uint32_t)dst_rank) : 0u;
     const uint32_t bbar = issuer ? mapa_rank(smem_addr(&sm.full[0]), (uint32_t)dst_rank) : 0u;
+    // TS: a label's value goes from its own lanes to every CTA by st.async
+    const uint32_t xg = smem_addr(&sm.gath[rank * CgE + (ro.lab_ok ? lc : 0)]), xb = smem_addr(&sm.full[0]);
     double(&Er)[CPL] = *reinterpret_cast<double(*)[CPL]>(&R[0]);
     double &W0 = R[0], &W1 = R[1], &V1 = R[2], &V2 = R[3], &pre = R[4], &gg = R[5], &pbe = R[6], &w0e = R[7],
            &coef = R[8], &a2 = R[9], &mu_acc = R[10], &musum = R[11], &bp = R[12], &start = R[13];
@@ -1097,10 +1109,10 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
     if constexpr (CLUSTER) cluster_barrier();
     else __syncthreads();
     if (ts) {   // bp[L-1] from the owners, later ones from the transition lanes (as forward)
-        if (own) sm.stage[lc] = fma(V1, w0e, pbe);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncthreads();
-        if (issuer) bulk_to_peer(bdst, smem_addr(sm.stage), (uint32_t)(CgE * 8), bbar);
+        if (own) {
+            const double b0 = fma(V1, w0e, pbe);
+            for (int dr = 0; dr < g.G; ++dr) st_async_at(mapa_rank(xg, dr), mapa_rank(xb, dr), b0);
+        }
     }
 
     int sK = (L - 1) % K;   // s mod K
@@ -1191,7 +1203,7 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
         } else if (ro.is_tr) {
             // ------------------------------------------- transposed transition
             if constexpr (CLUSTER) {
-                if (tid == 32 * g.NWO) mbar_expect_tx(&sm.full[par], g.G * (int)even_up(Cg) * 8);   // as forward
+                if (tid == 32 * g.NWO) mbar_expect_tx(&sm.full[par], ts ? C * 8 : g.G * (int)even_up(Cg) * 8);   // as forward
                 if (!ts) {
                     cta_barrier(5, NOT);   // the owners' stage is written
                     if (issuer)
@@ -1212,14 +1224,10 @@ __device__ __forceinline__ void cl_bwd_body(const FbArgs &a, const ClGeom &g, in
             group_sum2(q, n, g.LPL);
             if (ts) {
                 cta_barrier(kBarPub, NOT);
-                if (s >= 1) {   // bp[s-1] = (q_s gg_s) (W0 eb) + pre eb, staged and sent (as forward)
-                    if (ro.lab_ok && j == 0)
-                        sm.stage[(par ^ 1) * CgE + lc] = fma(q * sm.pub[lc], sm.pub[CgE + lc], sm.pub[2 * CgE + lc]);
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    cta_barrier(5, 32 * g.NWT);
-                    if (issuer)
-                        bulk_to_peer(bdst + (par ^ 1) * g.GP * 8, smem_addr(sm.stage + (par ^ 1) * CgE),
-                                     (uint32_t)(CgE * 8), bbar + (par ^ 1) * 8);
+                if (s >= 1 && ro.lab_ok) {   // bp[s-1] = (q_s gg_s) (W0 eb) + pre eb, sent (as forward)
+                    const double bn = fma(q * sm.pub[lc], sm.pub[CgE + lc], sm.pub[2 * CgE + lc]);
+                    const uint32_t og = xg + (uint32_t)((par ^ 1) * g.GP * 8), ob = xb + (uint32_t)((par ^ 1) * 8);
+                    for (int dr = j; dr < g.G; dr += g.LPL) st_async_at(mapa_rank(og, dr), mapa_rank(ob, dr), bn);
                 }
             }
             if (ro.lab_ok && j == 0) sm.qbuf[par * CgE + lc] = q;
