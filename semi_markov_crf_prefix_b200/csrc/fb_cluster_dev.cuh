@@ -393,6 +393,15 @@ __device__ __forceinline__ double window_bwd(double *ring, const double *Wd, int
     return strided_dot(ring + (size_t)(sK + i0) * RS + lc, step, Wd + (size_t)(i0 + 1) * RS + lc, step, n);
 }
 
+// A zero the compiler cannot see through, computed from v: adding it to an
+// address makes the loads from that address wait for v.
+__device__ __forceinline__ int opaque_zero(double v)
+{
+    int z;
+    asm("and.b32 %0, %1, 0;" : "=r"(z) : "r"((int)__double_as_longlong(v)));
+    return z;
+}
+
 // The same window sums with the lane's weights in registers (W[m] for row m of
 // the lane, 0 past the last duration) and no per-row bounds: NR rows per lane
 // (a bucket >= the rows the lane has), the rows beyond the window read the
@@ -411,8 +420,18 @@ __device__ __forceinline__ double window_fwd_reg(double *ring, int K, int RS, in
     const double *p = ring + (tauK + K - d0) * RS + lc;
     const int step = LPW * RS;
     double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    // eight rows at a time, each chunk's loads after the previous chunk's products:
+    // at most eight loads of a lane in the shared-memory queue, so the chain's own
+    // loads (the owners' q) do not wait behind a whole window pass
 #pragma unroll
-    for (int m = 0; m < NR; ++m) acc[m & 7] = fma(p[-m * step], W[m], acc[m & 7]);
+    for (int m0 = 0; m0 < NR; m0 += 8) {
+        double v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = p[-(m0 + i) * step];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fma(v[i], W[m0 + i], acc[i]);
+        if (m0 + 8 < NR) p += opaque_zero(acc[7]);
+    }
     return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
@@ -428,7 +447,14 @@ __device__ __forceinline__ double window_bwd_reg(double *ring, int K, int RS, in
     const int step = LPW * RS;
     double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-    for (int m = 0; m < NR; ++m) acc[m & 7] = fma(p[m * step], W[m], acc[m & 7]);
+    for (int m0 = 0; m0 < NR; m0 += 8) {   // eight rows at a time (as forward)
+        double v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = p[(m0 + i) * step];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fma(v[i], W[m0 + i], acc[i]);
+        if (m0 + 8 < NR) p += opaque_zero(acc[7]);
+    }
     return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
