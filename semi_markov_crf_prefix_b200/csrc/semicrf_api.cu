@@ -113,7 +113,10 @@ bool make_layout(const semicrf_dims &d, int what, const Plan &p, Layout *out)
     L.delta = d.ckpt_interval > 0 ? d.ckpt_interval : default_delta(d.T);
     if (L.delta > d.T) L.delta = d.T;
     L.J = (d.T + L.delta - 1) / L.delta;
-    int nch = (296 + d.B - 1) / d.B;
+    // prefix-scan chunks: eight CTAs per SM over the batch, so that the two
+    // HBM-bound passes keep enough loads in flight (two per SM left them at
+    // about half the copy bandwidth)
+    int nch = (8 * device_sm_count() + d.B - 1) / d.B;
     int maxch = (d.T + 63) / 64;
     if (nch > maxch) nch = maxch;
     if (nch < 1) nch = 1;
