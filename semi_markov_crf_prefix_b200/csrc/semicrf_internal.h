@@ -142,16 +142,19 @@ struct FbArgs {
 // when LPW > 32).
 // RS is the shared-memory row stride (doubles) of the ring, duration-weight and
 // duration-accumulator arrays, chosen so that the 16 lanes of a half-warp's
-// window loads (16/LPW labels x LPW consecutive rows) fall in distinct banks.  GP is the pitch of the exchanged
-// values: G blocks of Cg labels each padded to an even count (16-byte units for
-// the bulk copies), zeros in the padding and past the last block, at least the
-// positions the transition lanes read, so they read without bounds tests.
+// window loads (16/LPW labels x LPW consecutive rows) fall in distinct banks.
+// GP is the pitch of the exchanged values: G blocks of Cg labels each padded to
+// an even count (16-byte units for the owners' bulk copies), zeros in the
+// padding and past the last block, at least the positions the transition lanes
+// read, so they read without bounds tests.
 // NRB: rows per window lane read with the weights in registers (8, 16 or 32;
 // 0: the weights stay in shared memory); PAD: zero ring rows before and after
 // the ring for the rows a window lane reads past the window.  TS (clusters): 1 =
-// the transition lanes form and send each position's value as soon as their sum
-// is done (plans with at least four transition warps, where the sum is long and
-// there are enough warps to issue the copies); 0 = the owners form and send it.
+// the transition lanes form each position's value as soon as their sum is done
+// and store it into every CTA with st.async, and all window lanes share the
+// rescale of rebased labels (plans with at least four transition warps: many
+// labels per CTA, a long sum); 0 = the owners form the value and bulk-copy it,
+// and each label's window lanes rescale its rows.
 struct ClGeom {
     int G = 0, Cg = 0, LPL = 0, CPL = 0, LPW = 0, PW = 0, NWO = 0, NWT = 0, NWW = 0, NT = 0, RS = 0, GP = 0;
     int NRB = 0, PAD = 0, TS = 0;
